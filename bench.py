@@ -1,0 +1,467 @@
+"""Benchmark of the fused-attention hot path on B200.
+
+One step = one pass of every operation on the path over its own seeded,
+HBM-resident synthetic input:
+  prefill   Llama-3-8B-shaped causal prefill   B1 Hq32 Hkv8 S4096 D128  (frt_attn_fwd)
+  paged     paged GQA decode                   B4 Hq64 Hkv8 D128 ps16, lens U[1024,32768]
+                                               (frt_attn_decode_paged, fused LSE merge)
+  long      long-context split-KV decode       B1 Hq32 Hkv4 Skv262144 D128 ps16
+  contig    single-token GQA decode            B1 Hq32 Hkv8 Skv4096 D128 (frt_attn_fwd, Sq=1)
+Each step's working set (~0.9 GB) exceeds the 126 MB L2, and every call's
+inputs are evicted by the calls before it, so no call starts L2-warm.
+
+Prints ONE JSON line (rank 0).  `value` is whole-job steps per second; the
+per-call microseconds, TFLOP/s, GB/s and roofline fractions are under
+"calls"; "roofline" describes the dominant kernel.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (fp64, OpenMP) on the host cores on a
+bounded sample of the same step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from flash_attention_tiled_b200 import inputs  # noqa: E402
+
+METRIC = ("attn prefill TFLOP/s & decode KV GB/s vs B200 roofline; "
+          "µs/call at batch 1")
+WORKLOAD = ("llama3-8b causal prefill 4k (B1 Hq32 Hkv8 D128) + paged GQA decode "
+            "(B4 Hq64 Hkv8 D128 ps16 lens U[1024,32768]) + 256k split-KV decode "
+            "(B1 Hq32 Hkv4 D128 ps16) + 4k GQA decode (B1 Hq32 Hkv8 D128)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------- work figures
+def prefill_flops(w) -> float:
+    """4*D flops per visible (query, key) pair per query head (2 for Q.K^T,
+    2 for P.V; exp not counted); masked pairs are not counted."""
+    off = w.Skv - w.Sq
+    if w.causal:
+        pairs = sum(max(0, min(w.Skv, i + off + 1)) for i in range(w.Sq))
+    else:
+        pairs = w.Sq * w.Skv
+    return 4.0 * w.D * pairs * w.Hq * w.B
+
+
+def prefill_bytes(w) -> float:
+    q = w.B * w.Hq * w.Sq * w.D * 2
+    kv = 2 * w.B * w.Hkv * w.Skv * w.D * 2
+    return q + kv + q + w.B * w.Hq * w.Sq * 4          # Q, K, V, O, LSE
+
+
+def decode_bytes(B, Hq, Hkv, D, total_tokens) -> float:
+    """K and V of every cached token read once per KV head, plus q, o, lse."""
+    return 2.0 * total_tokens * Hkv * D * 2 + B * Hq * D * 2 * 2 + B * Hq * 4
+
+
+def decode_flops(Hq, D, total_tokens) -> float:
+    return 4.0 * D * Hq * total_tokens
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -------------------------------------------------------------- our arm
+class Step:
+    """The four calls of one step, with inputs resident on the device."""
+
+    def __init__(self, device):
+        from flash_attention_tiled_b200 import frt
+        self.frt = frt
+        self.dev = device
+        W = inputs.WORKLOADS
+        self.w_pf = W["llama3_8b_prefill_4k"]
+        self.w_pg = W["paged_gqa_decode_b4"]
+        self.w_lg = W["long_splitkv_decode_256k"]
+        self.w_ct = W["gqa_decode_4k"]
+        self.host = {
+            "prefill": inputs.make(self.w_pf),
+            "paged": inputs.make(self.w_pg),
+            "long": inputs.make(self.w_lg),
+            "contig": inputs.make(self.w_ct),
+        }
+        self.d = {k: {n: (t.to(device) if isinstance(t, torch.Tensor) else t)
+                      for n, t in v.items()} for k, v in self.host.items()}
+        self.tokens_pg = int(self.host["paged"]["seq_lens"].sum())
+        self.tokens_lg = int(self.host["long"]["seq_lens"].sum())
+        # outputs, allocated once
+        self.out = {
+            "prefill": (torch.empty_like(self.d["prefill"]["q"]),
+                        torch.empty(self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq, device=device)),
+            "paged": (torch.empty_like(self.d["paged"]["q"]),
+                      torch.empty(self.w_pg.B, self.w_pg.Hq, device=device)),
+            "long": (torch.empty_like(self.d["long"]["q"]),
+                     torch.empty(self.w_lg.B, self.w_lg.Hq, device=device)),
+            "contig": (torch.empty_like(self.d["contig"]["q"]),
+                       torch.empty(self.w_ct.B, self.w_ct.Hq, 1, device=device)),
+        }
+
+    def call(self, name, d=None, out=None):
+        d = self.d[name] if d is None else d
+        o, l = self.out[name] if out is None else out
+        f = self.frt
+        if name == "prefill":
+            f.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=self.w_pf.scale, out=o, lse=l)
+        elif name == "contig":
+            f.attn_fwd(d["q"], d["k"], d["v"], causal=False, scale=self.w_ct.scale, out=o, lse=l)
+        else:
+            w = self.w_pg if name == "paged" else self.w_lg
+            f.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
+                                d["seq_lens"], scale=w.scale, out=o, lse=l)
+
+    NAMES = ("prefill", "paged", "long", "contig")
+
+    def work(self):
+        """Algorithmic (flops, bytes) of each call."""
+        pf = self.w_pf
+        return {
+            "prefill": (prefill_flops(pf), prefill_bytes(pf)),
+            "paged": (decode_flops(self.w_pg.Hq, 128, self.tokens_pg),
+                      decode_bytes(self.w_pg.B, self.w_pg.Hq, self.w_pg.Hkv, 128, self.tokens_pg)),
+            "long": (decode_flops(self.w_lg.Hq, 128, self.tokens_lg),
+                     decode_bytes(1, self.w_lg.Hq, self.w_lg.Hkv, 128, self.tokens_lg)),
+            "contig": (decode_flops(self.w_ct.Hq, 128, self.w_ct.Skv),
+                       decode_bytes(1, self.w_ct.Hq, self.w_ct.Hkv, 128, self.w_ct.Skv)),
+        }
+
+
+def run_ours(args, rank, world, local_rank):
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    st = Step(device)
+    stream = torch.cuda.current_stream(device)
+    names = Step.NAMES
+    for _ in range(args.warmup):
+        for n in names:
+            st.call(n)
+    torch.cuda.synchronize(device)
+
+    # per-call events over the whole timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    with sampler:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            e = ev[s]
+            e[0].record(stream)
+            for i, n in enumerate(names):
+                st.call(n)
+                e[i + 1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    per_call_ms = {n: float(np.mean([ev[s][i].elapsed_time(ev[s][i + 1])
+                                     for s in range(args.steps)]))
+                   for i, n in enumerate(names)}
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(st, args, device)
+
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    work = st.work()
+    calls = {}
+    for n in names:
+        fl, by = work[n]
+        us = per_call_ms[n] * 1e3
+        rec = {"us": round(us, 2), "tflops": round(fl / us * 1e-6, 1),
+               "gbs": round(by / us * 1e-3, 1)}
+        if n == "prefill":
+            rec["bound"] = "tensor"
+            rec["frac"] = round(rec["tflops"] / peaks["bf16_tflops"], 4)
+        else:
+            rec["bound"] = "hbm"
+            rec["frac"] = round(rec["gbs"] / peaks["hbm_gbs"], 4)
+        calls[n] = rec
+    dom = max(names, key=lambda n: per_call_ms[n])
+    d = calls[dom]
+    if d["bound"] == "tensor":
+        roof = {"bound": "tensor", "achieved": d["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} (burst figure: each kernel runs < 1 ms)"
+    roof["traffic"] = None
+
+    cpu = cpu_baseline(st, per_step_only=True)
+    line = {
+        "metric": METRIC,
+        "value": round(world * args.steps / (total_ms * 1e-3), 2),
+        "unit": "step/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, shuffled page tables)",
+        "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "working set per step ~0.9 GB > 126 MB L2; each call's inputs are "
+                         "evicted by the calls before it (no explicit flush)"},
+        "calls": calls,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": len(names) * args.steps,
+        "clocks": sampler.summary(),
+    }
+    return line
+
+
+def run_e2e(st: Step, args, device):
+    """Same step through the public API with pinned host inputs: H2D copy of
+    every call's inputs, the call, and a D2H read of its outputs, per step."""
+    names = Step.NAMES
+    host = {n: {k: (t.pin_memory() if isinstance(t, torch.Tensor) else t)
+                for k, t in st.host[n].items()} for n in names}
+    outs_h = {n: tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in st.out[n])
+              for n in names}
+    scratch = {n: {k: torch.empty_like(t) if isinstance(t, torch.Tensor) else t
+                   for k, t in st.d[n].items()} for n in names}
+    h2d = sum(t.numel() * t.element_size() for n in names for t in host[n].values()
+              if isinstance(t, torch.Tensor))
+    d2h = sum(t.numel() * t.element_size() for n in names for t in outs_h[n])
+    stream = torch.cuda.current_stream(device)
+    steps = max(1, min(args.steps, 10))
+
+    def one():
+        for n in names:
+            for k, t in host[n].items():
+                if isinstance(t, torch.Tensor):
+                    scratch[n][k].copy_(t, non_blocking=True)
+            st.call(n, d=scratch[n])
+            for h, dv in zip(outs_h[n], st.out[n]):
+                h.copy_(dv, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    return {"value": round(1e3 / ms, 3), "unit": "step/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3), "steps": steps}
+
+
+# ------------------------------------------------------------- oracle arm
+def cpu_sample_plan():
+    """Bounded oracle sample of one step and the factor scaling it to a full step:
+    prefill on 8 of 32 query heads (full causal rows), paged decode on 16 of
+    256 rows, long decode on 4 of 32 heads, contiguous decode on all 32 heads."""
+    return {"prefill_heads": 8, "paged_rows": 16, "long_heads": 4}
+
+
+def cpu_baseline(st: Step | None, per_step_only=False, host=None):
+    import oracle
+    plan = cpu_sample_plan()
+    W = inputs.WORKLOADS
+    if host is None:
+        host = st.host
+    t_total = 0.0
+    t0 = time.perf_counter()
+    # prefill: the first `prefill_heads` query heads with their KV heads
+    w = W["llama3_8b_prefill_4k"]
+    x = host["prefill"]
+    hq = plan["prefill_heads"]
+    g = w.Hq // w.Hkv
+    hkv = (hq + g - 1) // g
+    ts = time.perf_counter()
+    oracle.attn_fwd(x["q"][:, :hq].contiguous(), x["k"][:, :hkv].contiguous(),
+                    x["v"][:, :hkv].contiguous(), True, w.scale)
+    t_total += (time.perf_counter() - ts) * (w.Hq / hq)
+    # paged decode: a mask of rows
+    for name, key, rows_key in (("paged_gqa_decode_b4", "paged", "paged_rows"),
+                                ("long_splitkv_decode_256k", "long", "long_heads")):
+        w = W[name]
+        x = host[key]
+        n_rows = plan[rows_key]
+        mask = np.zeros((w.B, w.Hq), dtype=bool)
+        mask.reshape(-1)[:n_rows] = True
+        ts = time.perf_counter()
+        oracle.attn_decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"],
+                                 x["seq_lens"], w.scale, heads_mask=mask)
+        t_total += (time.perf_counter() - ts) * (w.B * w.Hq / n_rows)
+    w = W["gqa_decode_4k"]
+    x = host["contig"]
+    ts = time.perf_counter()
+    oracle.attn_fwd(x["q"], x["k"], x["v"], False, w.scale)
+    t_total += time.perf_counter() - ts
+    wall = time.perf_counter() - t0
+    return {"value": round(1.0 / t_total, 6), "unit": "step/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": (f"one step sampled: prefill {plan['prefill_heads']}/32 heads, paged "
+                       f"decode {plan['paged_rows']}/256 rows, long decode "
+                       f"{plan['long_heads']}/32 heads, contiguous decode all 32 heads; "
+                       f"each leg's time scaled by its sampled fraction "
+                       f"({wall:.1f} s of CPU wall time)"),
+            "s_per_step": round(t_total, 3)}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    host = {"prefill": inputs.make("llama3_8b_prefill_4k"), "paged": inputs.make("paged_gqa_decode_b4"),
+            "long": inputs.make("long_splitkv_decode_256k"), "contig": inputs.make("gqa_decode_4k")}
+    for _ in range(args.warmup_ref):
+        cpu_baseline(None, host=host)
+    vals = [cpu_baseline(None, host=host) for _ in range(args.steps_ref)]
+    s_per_step = float(np.mean([v["s_per_step"] for v in vals]))
+    cb = vals[-1]
+    value = round(1.0 / s_per_step, 6)
+    cb["value"] = value
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "step/s", "n_gpus": 1,
+        "steps": args.steps_ref, "warmup": args.warmup_ref,
+        "ms_per_step": round(s_per_step * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, shuffled page tables)",
+        "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "step/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # each oracle step is a bounded sample of ~10 s; keep the run to minutes
+        args.steps_ref = max(1, min(args.steps, 3))
+        args.warmup_ref = 0
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

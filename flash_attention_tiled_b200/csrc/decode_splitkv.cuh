@@ -1,0 +1,501 @@
+// decode_splitkv.cuh -- split-KV decode attention (one query token per
+// sequence) over a paged or contiguous KV cache, for sm_100a.
+//
+// What it computes: softmax attention of each query head over its sequence's
+// cached keys, as the online-softmax kernel of the "Real-time inference
+// optimisation" page (llmapi-app.pages.dev, section "Flash Attention
+// optimisation") does, over a KV cache cut into 16-token pages (same page,
+// method paged_attention), with MQA/GQA head sharing ("FlashRT-HF-kernels"
+// page, section "Attention optimisation").  Partial results over disjoint
+// key ranges are combined by their log-sum-exp, the correct form of that
+// page's per-page sum.
+//
+// Work plan (flattened split-KV).  A segment is (sequence b, KV head kvh,
+// group of up to 16 query heads of that KV head); it owns ceil(len_b/16)
+// pages.  All segments' pages are laid end to end (units) and the CTAs of the
+// grid take equal contiguous shares of that line, so every CTA streams the
+// same number of pages whatever the length mix.  The piece of a segment that
+// falls inside one CTA is reduced to one partial (o, lse); a segment wholly
+// inside one CTA is written out directly, otherwise the last CTA to finish
+// one of its pieces merges all of them by log-sum-exp (an atomic ticket per
+// segment; no CTA ever waits for another).
+//
+// Inside a CTA: warp 0 streams pages into a ring of shared-memory stages with
+// TMA (128-byte swizzled 16x64 boxes, one mbarrier per stage), looking pages
+// up in the block table; warps 1..W each take one page of every stage and
+// compute S = Q.K^T and O += P.V with warp-level bf16 MMAs in which the
+// segment's query heads form the M dimension, so each K/V page is read from
+// HBM once for all heads of its group.  Scores live in the exp2 domain
+// (scale * log2(e) folded in); the online max/sum use quad shuffles.
+#pragma once
+
+#include "frt_device.cuh"
+
+namespace frt {
+
+constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
+constexpr int kDecWarps = 4;          // consumer warps per CTA
+constexpr int kDecThreads = 32 * (kDecWarps + 1);
+constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
+constexpr int kDecMaxBatch = 1024;    // prefix table held in shared memory
+
+struct DecodeParams {
+  const __nv_bfloat16* q;        // [B, Hq, D]
+  __nv_bfloat16* o;              // [B, Hq, D]
+  float* lse;                    // [B, Hq] natural log, or nullptr
+  const int32_t* block_table;    // paged: [B, max_pages]; contiguous: nullptr
+  const int32_t* seq_lens;       // paged: [B] (device); contiguous: nullptr
+  int max_pages;                 // paged: block-table row length
+  int contig_len;                // contiguous: keys per sequence (Skv)
+  int B, Hq, Hkv, g, hgroups;    // g = Hq / Hkv, hgroups = ceil(g / 16)
+  float scale_log2;              // scale * log2(e)
+  float* ws_o;                   // [slots, 16, D] fp32 partial outputs (normalised)
+  float* ws_lse;                 // [slots, 16] fp32 partial LSE (log2 domain)
+  unsigned* ws_count;            // [segments] arrival tickets, zero between calls
+};
+
+template <int D>
+struct DecodeSmem {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 64 bf16
+  static constexpr int kPageBytes = kHalves * kBoxBytes;              // K or V of one page
+  static constexpr int kStageBytes = kDecWarps * 2 * kPageBytes;      // K+V of W pages
+  static constexpr int kStages = (D == 128) ? 5 : 10;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  // cross-warp merge scratch: per warp m[16], l[16], l_exact[16], O[16][D]
+  static constexpr int kScratchStride = 3 * kDecHeadsPerSeg + kDecHeadsPerSeg * D;
+  static constexpr int kScratchFloats = kDecWarps * kScratchStride;
+  static constexpr int kScratchOff = kRingBytes;
+  static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
+  static constexpr int kBarOff = kPrefixOff + ((kDecMaxBatch + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kBytes = 1024 /*alignment slack*/ + kBarOff + 2 * kStages * 8;
+  static_assert(kBarOff % 8 == 0, "mbarriers need 8-byte alignment");
+};
+
+// Pages of sequence b (seq_len clamped to [0, max_pages * 16]).
+__device__ __forceinline__ int dec_pages_of(const DecodeParams& p, int b) {
+  if (p.seq_lens == nullptr) return (p.contig_len + kDecPage - 1) / kDecPage;
+  int len = p.seq_lens[b];
+  len = len < 0 ? 0 : len;
+  long long cap = (long long)p.max_pages * kDecPage;
+  if (len > cap) len = (int)cap;
+  return (len + kDecPage - 1) / kDecPage;
+}
+
+__device__ __forceinline__ int dec_len_of(const DecodeParams& p, int b) {
+  if (p.seq_lens == nullptr) return p.contig_len;
+  int len = p.seq_lens[b];
+  len = len < 0 ? 0 : len;
+  long long cap = (long long)p.max_pages * kDecPage;
+  return len > cap ? (int)cap : len;
+}
+
+// CTA whose share of the unit line [0, T) holds unit u (shares are
+// [floor(c*T/C), floor((c+1)*T/C)); requires T >= C so none is empty).
+__device__ __forceinline__ int dec_cta_of(long long u, long long T, int C) {
+  return (int)(((u + 1) * (long long)C - 1) / T);
+}
+
+// Swizzled shared-memory address of the 16-byte chunk holding element
+// (row, col) of a 16 x 64 bf16 TMA box written with 128-byte swizzling.
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t box_base, int row, int col) {
+  return box_base + row * 128 + ((((col >> 3) ^ (row & 7))) << 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  using L = DecodeSmem<D>;
+  constexpr int kHalves = L::kHalves;
+  constexpr int kStages = L::kStages;
+  constexpr int kKSteps = D / 16;     // MMA K-steps of Q.K^T
+  constexpr int kNTiles = D / 8;      // 8-wide output tiles of P.V
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  float* scratch = reinterpret_cast<float*>(smem + L::kScratchOff);
+  int* prefix = reinterpret_cast<int*>(smem + L::kPrefixOff);   // [B+1] page prefix
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty_bar = full_bar + kStages;
+  __shared__ int abort_flag;
+  __shared__ int s_is_last;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int nseg_b = p.Hkv * p.hgroups;   // segments per sequence
+
+  // ---- per-sequence page prefix (warp 0: chunked scan), barriers
+  if (warp == 0) {
+    const int per = (p.B + 31) / 32;
+    const int b0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (b0 + i < p.B) local += dec_pages_of(p, b0 + i);
+    int incl = local;
+    for (int off = 1; off < 32; off <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int i = 0; i < per; ++i)
+      if (b0 + i < p.B) {
+        prefix[b0 + i] = run;
+        run += dec_pages_of(p, b0 + i);
+      }
+    if (lane == 31) prefix[p.B] = incl;
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&full_bar[s], 1);
+        mbar_init(&empty_bar[s], kDecWarps);
+      }
+      abort_flag = 0;
+      fence_barrier_init();
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+    }
+  }
+  __syncthreads();
+
+  const long long T = (long long)prefix[p.B] * nseg_b;   // total units
+  const int C = (int)min((long long)gridDim.x, T);       // CTAs with a non-empty share
+  const int c = blockIdx.x;
+
+  // ---- sequences with no key: o = 0, lse = -inf (spread over the grid)
+  for (int b = c; b < p.B; b += gridDim.x) {
+    if (prefix[b + 1] != prefix[b]) continue;
+    for (int i = threadIdx.x; i < p.Hq * D; i += blockDim.x)
+      p.o[(size_t)b * p.Hq * D + i] = __float2bfloat16(0.f);
+    if (p.lse != nullptr)
+      for (int i = threadIdx.x; i < p.Hq; i += blockDim.x) p.lse[(size_t)b * p.Hq + i] = -INFINITY;
+  }
+  if (c >= C) return;
+
+  const long long u_begin = (long long)c * T / C;
+  const long long u_end = (long long)(c + 1) * T / C;
+
+  // Walk of this CTA's pieces, identical in every warp.  Returns false when
+  // the share is exhausted.  (b, seg_in_b) identify the segment, pages
+  // [pg0, pg1) of it lie in this CTA, npg = pages of the segment.
+  struct Piece {
+    int b, seg_in_b, pg0, pg1, npg;
+    long long seg_u0;
+  };
+  auto first_piece = [&](Piece& pc) {
+    // largest b with prefix[b] * nseg_b <= u_begin and a non-empty sequence
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if ((long long)prefix[mid] * nseg_b <= u_begin) lo = mid; else hi = mid - 1;
+    }
+    int b = lo;
+    while (prefix[b + 1] == prefix[b]) ++b;   // skip empty sequences
+    const int npg = prefix[b + 1] - prefix[b];
+    const long long off = u_begin - (long long)prefix[b] * nseg_b;
+    pc.b = b;
+    pc.seg_in_b = (int)(off / npg);
+    pc.npg = npg;
+    pc.seg_u0 = (long long)prefix[b] * nseg_b + (long long)pc.seg_in_b * npg;
+    pc.pg0 = (int)(off % npg);
+    long long seg_end = pc.seg_u0 + npg;
+    pc.pg1 = (int)((seg_end < u_end ? seg_end : u_end) - pc.seg_u0);
+  };
+  auto next_piece = [&](Piece& pc) -> bool {
+    long long u = pc.seg_u0 + pc.pg1;
+    if (u >= u_end) return false;
+    int b = pc.b, s = pc.seg_in_b + 1;
+    if (s == nseg_b) {
+      s = 0;
+      ++b;
+      while (prefix[b + 1] == prefix[b]) ++b;
+    }
+    const int npg = prefix[b + 1] - prefix[b];
+    pc.b = b;
+    pc.seg_in_b = s;
+    pc.npg = npg;
+    pc.seg_u0 = u;
+    pc.pg0 = 0;
+    pc.pg1 = (int)((u + npg < u_end ? u + npg : u_end) - u);
+    return true;
+  };
+
+  if (warp == 0) {
+    // =================================================== producer (TMA)
+    int stage = 0;
+    uint32_t phase = 0;
+    Piece pc;
+    first_piece(pc);
+    bool ok = true;
+    do {
+      const int kvh = pc.seg_in_b / p.hgroups;
+      for (int pb = pc.pg0; pb < pc.pg1 && ok; pb += kDecWarps) {
+        const int n = min(kDecWarps, pc.pg1 - pb);
+        // row of the page's first token in the [rows, D] view of the cache
+        int row = 0;
+        if (lane < n) {
+          const int page = pb + lane;
+          if (p.block_table != nullptr) {
+            const int phys = p.block_table[(size_t)pc.b * p.max_pages + page];
+            row = (phys * p.Hkv + kvh) * kDecPage;
+          } else {
+            row = ((pc.b * p.Hkv + kvh) * p.contig_len) + page * kDecPage;
+          }
+        }
+        ok = mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], n * 2 * L::kPageBytes);
+        __syncwarp();
+        if (lane < n) {
+          uint8_t* kdst = ring + stage * L::kStageBytes + lane * 2 * L::kPageBytes;
+          uint8_t* vdst = kdst + L::kPageBytes;
+#pragma unroll
+          for (int h = 0; h < kHalves; ++h) {
+            tma_load_2d(kdst + h * L::kBoxBytes, &tmap_k, &full_bar[stage], h * 64, row);
+            tma_load_2d(vdst + h * L::kBoxBytes, &tmap_v, &full_bar[stage], h * 64, row);
+          }
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    } while (ok && next_piece(pc));
+    // Normal exit needs no drain: the consumers wait for every stage issued
+    // here before the CTA can finish.  After an abort they may not, so give
+    // copies still in flight time to land before this warp leaves.
+    if (!ok) __nanosleep(100000);
+    return;
+  }
+
+  // ====================================================== consumers (MMA)
+  const int cw = warp - 1;               // consumer warp index
+  const int quad = lane >> 2;            // MMA row group: head rows quad, quad+8
+  const int qc = lane & 3;               // column pair within the quad
+  float* my_m = scratch + cw * L::kScratchStride;
+  float* my_l = my_m + kDecHeadsPerSeg;
+  float* my_le = my_l + kDecHeadsPerSeg;
+  float* my_o = my_le + kDecHeadsPerSeg;
+  const uint32_t ring_u32 = smem_u32(ring);
+
+  int stage = 0;
+  uint32_t phase = 0;
+  Piece pc;
+  first_piece(pc);
+  bool ok = true;
+  do {
+    const int kvh = pc.seg_in_b / p.hgroups;
+    const int hg = pc.seg_in_b % p.hgroups;
+    const int h0 = kvh * p.g + hg * kDecHeadsPerSeg;            // first query head
+    const int nh = min(kDecHeadsPerSeg, p.g - hg * kDecHeadsPerSeg);
+    const int len = dec_len_of(p, pc.b);
+
+    // Q fragments (A operand, row = head, col = d), rows >= nh are zero
+    uint32_t qa[kKSteps][4];
+    {
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)pc.b * p.Hq + h0) * D);
+#pragma unroll
+      for (int ks = 0; ks < kKSteps; ++ks) {
+        const int c0 = ks * 16 + 2 * qc;
+        qa[ks][0] = quad < nh ? q32[(quad * D + c0) / 2] : 0u;
+        qa[ks][1] = quad + 8 < nh ? q32[((quad + 8) * D + c0) / 2] : 0u;
+        qa[ks][2] = quad < nh ? q32[(quad * D + c0 + 8) / 2] : 0u;
+        qa[ks][3] = quad + 8 < nh ? q32[((quad + 8) * D + c0 + 8) / 2] : 0u;
+      }
+    }
+    float m_run[2] = {-INFINITY, -INFINITY};   // rows quad, quad+8 (exp2 domain)
+    float l_run[2] = {0.f, 0.f};     // this lane's share of the rounded-weight row sums
+    float le_run[2] = {0.f, 0.f};    // and of the exact-weight row sums (for the LSE)
+    float acc[kNTiles][4];
+#pragma unroll
+    for (int t = 0; t < kNTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+    for (int pb = pc.pg0; pb < pc.pg1; pb += kDecWarps) {
+      ok = mbar_wait_warp(&full_bar[stage], phase, &abort_flag);
+      if (!ok) break;
+      const int page = pb + cw;
+      if (page < pc.pg1) {
+        const uint32_t kbase = ring_u32 + stage * L::kStageBytes + cw * 2 * L::kPageBytes;
+        const uint32_t vbase = kbase + L::kPageBytes;
+        const int valid = min(kDecPage, len - page * kDecPage);   // tokens of this page
+
+        // ---- S = Q.K^T: two 16x8 tiles (tokens 0-7, 8-15)
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = (mi >> 1) * 8 + r;
+#pragma unroll
+          for (int ks = 0; ks < kKSteps; ++ks) {
+            const int col = ks * 16 + (mi & 1) * 8;
+            const uint32_t addr =
+                sw128_addr(kbase + (col >> 6) * L::kBoxBytes, tok, col & 63);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(addr, b0, b1, b2, b3);
+            mma_bf16_16816(s0, qa[ks], b0, b1);
+            mma_bf16_16816(s1, qa[ks], b2, b3);
+          }
+        }
+        // ---- scores in the exp2 domain, tail tokens masked by select
+        const int t0 = 2 * qc;   // token of s0[0]; s0[1] -> t0+1; s1 -> +8
+        float sc[2][4];          // [row half][tok t0, t0+1, t0+8, t0+9]
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          sc[rh][0] = (t0 < valid) ? s0[2 * rh] * p.scale_log2 : -INFINITY;
+          sc[rh][1] = (t0 + 1 < valid) ? s0[2 * rh + 1] * p.scale_log2 : -INFINITY;
+          sc[rh][2] = (t0 + 8 < valid) ? s1[2 * rh] * p.scale_log2 : -INFINITY;
+          sc[rh][3] = (t0 + 9 < valid) ? s1[2 * rh + 1] * p.scale_log2 : -INFINITY;
+        }
+        uint32_t pa[4];
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          float mx = fmaxf(fmaxf(sc[rh][0], sc[rh][1]), fmaxf(sc[rh][2], sc[rh][3]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float m_new = fmaxf(m_run[rh], mx);
+          const float alpha = fast_exp2(m_run[rh] - m_new);   // 0 on the first page
+          m_run[rh] = m_new;
+          const float e0 = fast_exp2(sc[rh][0] - m_new), e1 = fast_exp2(sc[rh][1] - m_new);
+          const float e2 = fast_exp2(sc[rh][2] - m_new), e3 = fast_exp2(sc[rh][3] - m_new);
+          const uint32_t lo = pack_bf16x2(e0, e1);
+          const uint32_t hi = pack_bf16x2(e2, e3);
+          // O is normalised by the bf16-rounded weights that feed P.V; the LSE
+          // uses the exact ones
+          const float psum = __uint_as_float(lo << 16) + __uint_as_float(lo & 0xffff0000u) +
+                             __uint_as_float(hi << 16) + __uint_as_float(hi & 0xffff0000u);
+          l_run[rh] = l_run[rh] * alpha + psum;
+          le_run[rh] = le_run[rh] * alpha + ((e0 + e1) + (e2 + e3));
+#pragma unroll
+          for (int t = 0; t < kNTiles; ++t) {
+            acc[t][2 * rh] *= alpha;
+            acc[t][2 * rh + 1] *= alpha;
+          }
+          pa[rh] = lo;        // a0a1 (rh=0) / a2a3 (rh=1): tokens t0, t0+1
+          pa[2 + rh] = hi;    // a4a5 / a6a7: tokens t0+8, t0+9
+        }
+        // ---- O += P.V: V^T fragments by transposing ldmatrix
+        {
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = (mi & 1) * 8 + r;
+          // B-fragment halves: b0b1 -> tokens 2qc, 2qc+1; b2b3 -> +8
+          const bool kill_lo0 = t0 >= valid, kill_hi0 = t0 + 1 >= valid;
+          const bool kill_lo1 = t0 + 8 >= valid, kill_hi1 = t0 + 9 >= valid;
+          const bool tail = valid < kDecPage;
+#pragma unroll
+          for (int nt = 0; nt < kNTiles; nt += 2) {
+            const int col = (nt + (mi >> 1)) * 8;
+            const uint32_t addr =
+                sw128_addr(vbase + (col >> 6) * L::kBoxBytes, tok, col & 63);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_trans(addr, b0, b1, b2, b3);
+            if (tail) {   // tokens past the sequence end may hold anything (NaN)
+              b0 = (kill_lo0 ? 0u : (b0 & 0xffffu)) | (kill_hi0 ? 0u : (b0 & 0xffff0000u));
+              b2 = (kill_lo0 ? 0u : (b2 & 0xffffu)) | (kill_hi0 ? 0u : (b2 & 0xffff0000u));
+              b1 = (kill_lo1 ? 0u : (b1 & 0xffffu)) | (kill_hi1 ? 0u : (b1 & 0xffff0000u));
+              b3 = (kill_lo1 ? 0u : (b3 & 0xffffu)) | (kill_hi1 ? 0u : (b3 & 0xffff0000u));
+            }
+            mma_bf16_16816(acc[nt], pa, b0, b1);
+            mma_bf16_16816(acc[nt + 1], pa, b2, b3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == kStages) { stage = 0; phase ^= 1u; }
+    }
+
+    // ---- this warp's state -> scratch
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+      float ls = l_run[rh], le = le_run[rh];
+      ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+      ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+      le += __shfl_xor_sync(0xffffffffu, le, 1);
+      le += __shfl_xor_sync(0xffffffffu, le, 2);
+      if (qc == 0) {
+        my_m[quad + 8 * rh] = m_run[rh];
+        my_l[quad + 8 * rh] = ls;
+        my_le[quad + 8 * rh] = le;
+      }
+#pragma unroll
+      for (int t = 0; t < kNTiles; ++t) {
+        float2 v2 = make_float2(acc[t][2 * rh], acc[t][2 * rh + 1]);
+        *reinterpret_cast<float2*>(&my_o[(quad + 8 * rh) * D + t * 8 + 2 * qc]) = v2;
+      }
+    }
+    // stop together if any warp gave up (every consumer gets the same answer)
+    if (bar_sync_or(1, kDecWarps * 32, !ok || abort_flag)) break;
+
+    // ---- combine the warps: one partial (or the final result) per piece
+    const int seg = pc.b * nseg_b + pc.seg_in_b;
+    const bool whole = (pc.pg0 == 0) && (pc.pg1 == pc.npg);
+    const int slot = c + seg;
+    const int ct = threadIdx.x - 32;
+    constexpr int kStride = L::kScratchStride;
+    for (int e = ct; e < nh * D; e += kDecWarps * 32) {
+      const int r = e / D, d = e % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, scratch[w * kStride + r]);
+      float Lsum = 0.f, Lexact = 0.f, Osum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float* sw = scratch + w * kStride;
+        const float mw = sw[r];
+        const float wgt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+        Lsum += wgt * sw[kDecHeadsPerSeg + r];
+        Lexact += wgt * sw[2 * kDecHeadsPerSeg + r];
+        Osum += wgt * sw[3 * kDecHeadsPerSeg + r * D + d];
+      }
+      const float o_val = Osum / Lsum;
+      const float lse2 = M + fast_log2(Lexact);
+      if (whole) {
+        const size_t row = (size_t)pc.b * p.Hq + h0 + r;
+        p.o[row * D + d] = __float2bfloat16(o_val);
+        if (d == 0 && p.lse != nullptr) p.lse[row] = lse2 * 0.69314718055994530942f;
+      } else {
+        p.ws_o[((size_t)slot * kDecHeadsPerSeg + r) * D + d] = o_val;
+        if (d == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
+      }
+    }
+    if (!whole) {
+      // ticket: the last piece of this segment to finish merges all of them
+      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
+      if (ct == 0) {
+        __threadfence();
+        const long long T_ = T;
+        const int c_first = dec_cta_of(pc.seg_u0, T_, C);
+        const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T_, C);
+        const unsigned parts = (unsigned)(c_last - c_first + 1);
+        const unsigned prev = atomicAdd(&p.ws_count[seg], 1u);
+        s_is_last = (prev == parts - 1) ? (c_first + 1) : 0;   // store c_first + 1
+        if (prev == parts - 1) {
+          p.ws_count[seg] = 0u;   // ready for the next call
+          __threadfence();
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
+      if (s_is_last) {
+        const int c_first = s_is_last - 1;
+        const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C);
+        for (int e = ct; e < nh * D; e += kDecWarps * 32) {
+          const int r = e / D, d = e % D;
+          float M = -INFINITY;
+          for (int cc = c_first; cc <= c_last; ++cc)
+            M = fmaxf(M, __ldcg(&p.ws_lse[(size_t)(cc + seg) * kDecHeadsPerSeg + r]));
+          float Lsum = 0.f, Osum = 0.f;
+          for (int cc = c_first; cc <= c_last; ++cc) {
+            const size_t sl = (size_t)(cc + seg);
+            const float wgt = fast_exp2(__ldcg(&p.ws_lse[sl * kDecHeadsPerSeg + r]) - M);
+            Lsum += wgt;
+            Osum += wgt * __ldcg(&p.ws_o[(sl * kDecHeadsPerSeg + r) * D + d]);
+          }
+          const size_t row = (size_t)pc.b * p.Hq + h0 + r;
+          p.o[row * D + d] = __float2bfloat16(Osum / Lsum);
+          if (d == 0 && p.lse != nullptr)
+            p.lse[row] = (M + fast_log2(Lsum)) * 0.69314718055994530942f;
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch reuse
+  } while (next_piece(pc));
+}
+
+}  // namespace frt

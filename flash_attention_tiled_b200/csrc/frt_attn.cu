@@ -1,0 +1,341 @@
+// frt_attn.cu -- the C ABI of the library (declared in include/frt_attn.h):
+// argument validation, work planning, TMA descriptor encoding and kernel
+// launches on the caller's stream.  This is the library's single translation
+// unit; the kernels live in the .cuh files it includes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/frt_attn.h"
+#include "decode_splitkv.cuh"
+#include "frt_device.cuh"
+#include "merge_lse.cuh"
+#include "prefill_sm100.cuh"
+
+namespace frt {
+
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------- device properties
+struct DeviceInfo {
+  int sm_count = 0;
+  bool kernels_configured = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+frt_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FRT_ERR_CUDA;
+  DeviceInfo& di = g_dev[dev];
+  if (!di.kernels_configured) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!di.kernels_configured) {
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FRT_ERR_CUDA;
+      di.sm_count = sms;
+      if (cudaFuncSetAttribute(decode_splitkv_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<128>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(decode_splitkv_kernel<64>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<64>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PrefillSmem<128>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PrefillSmem<64>::kBytes) != cudaSuccess)
+        return FRT_ERR_CUDA;
+      di.kernels_configured = true;
+    }
+  }
+  *out = &di;
+  return FRT_OK;
+}
+
+// ------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzling.  dims/box are innermost first;
+// strides_bytes[i] is the stride of dims[i + 1].
+bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estr[i] = 1;
+    if (i + 1 < rank) gstr[i] = strides_bytes[i];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool scale_ok(float scale) { return scale > 0.f && isfinite(scale); }
+
+// ---------------------------------------------------- decode workspace
+struct DecodeWorkspace {
+  size_t o_off, lse_off, count_off, total;
+};
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Counters first: their offset does not depend on the problem shape.
+DecodeWorkspace decode_ws_layout(long long parts, long long segments, int D) {
+  DecodeWorkspace w;
+  const long long slots = parts + segments;
+  w.count_off = 0;
+  w.lse_off = round_up((size_t)segments * sizeof(unsigned), 256);
+  w.o_off = w.lse_off + round_up((size_t)slots * kDecHeadsPerSeg * sizeof(float), 256);
+  w.total = w.o_off + round_up((size_t)slots * kDecHeadsPerSeg * D * sizeof(float), 256);
+  return w;
+}
+
+// Shared launcher of the split-KV decode kernel (paged or contiguous cache).
+frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
+                         uint64_t cache_rows, const int32_t* block_table, int max_pages,
+                         const int32_t* seq_lens, int contig_len, void* o, float* lse, int B,
+                         int Hq, int Hkv, int D, float scale, int num_splits, void* workspace,
+                         size_t* workspace_bytes, cudaStream_t stream) {
+  const bool query = (q == nullptr);
+  DeviceInfo* di = nullptr;
+  if (!query) {
+    frt_status st = device_info(&di);
+    if (st != FRT_OK) return st;
+  }
+  const int g = Hq / Hkv;
+  const int hgroups = (g + kDecHeadsPerSeg - 1) / kDecHeadsPerSeg;
+  const long long segments = (long long)B * Hkv * hgroups;
+  int parts = num_splits;
+  if (parts <= 0) {
+    if (di == nullptr) {
+      frt_status st = device_info(&di);
+      if (st != FRT_OK) return st;
+    }
+    parts = di->sm_count;
+  }
+  const DecodeWorkspace wl = decode_ws_layout(parts, segments, D);
+  if (query) {
+    if (workspace_bytes == nullptr) return FRT_ERR_INVALID_ARG;
+    *workspace_bytes = wl.total;
+    return FRT_OK;
+  }
+  if (B == 0) return FRT_OK;
+  if (workspace == nullptr || workspace_bytes == nullptr || *workspace_bytes < wl.total ||
+      !aligned16(workspace))
+    return FRT_ERR_WORKSPACE;
+
+  CUtensorMap tk, tv;
+  const uint64_t dims[2] = {(uint64_t)D, cache_rows};
+  const uint64_t strides[1] = {(uint64_t)D * 2};
+  const uint32_t box[2] = {64, (uint32_t)kDecPage};
+  if (!make_tmap(&tk, k_base, 2, dims, strides, box) ||
+      !make_tmap(&tv, v_base, 2, dims, strides, box))
+    return FRT_ERR_CUDA;
+
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.max_pages = max_pages;
+  p.contig_len = contig_len;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.g = g;
+  p.hgroups = hgroups;
+  p.scale_log2 = scale * kLog2e;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+  p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.ws_count = reinterpret_cast<unsigned*>(ws + wl.count_off);
+
+  if (D == 128)
+    decode_splitkv_kernel<128><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
+  else
+    decode_splitkv_kernel<64><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+// Tiled tensor-core forward (Sq > 1).
+frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
+                          float scale, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  frt_status st = device_info(&di);
+  if (st != FRT_OK) return st;
+  const int n_qtiles = (Sq + kPfBM - 1) / kPfBM;
+  if (n_qtiles > 65535) return FRT_ERR_UNSUPPORTED;
+  // With Skv == 0 every tile has no key tile to visit (o = 0, lse = -inf);
+  // the K/V maps then only need to be valid descriptors, never read.
+  const void* kb = Skv > 0 ? k : q;
+  const void* vb = Skv > 0 ? v : q;
+  const int skv_map = Skv > 0 ? Skv : 1;
+  CUtensorMap tq, tk, tv, to;
+  const uint32_t box[3] = {64, (uint32_t)kPfBM, 1};
+  const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * Hq};
+  const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
+  const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)skv_map,
+                             (uint64_t)(Skv > 0 ? B * Hkv : 1)};
+  const uint64_t kstr[2] = {(uint64_t)D * 2, (uint64_t)skv_map * D * 2};
+  if (!make_tmap(&tq, q, 3, qdims, qstr, box) || !make_tmap(&tk, kb, 3, kdims, kstr, box) ||
+      !make_tmap(&tv, vb, 3, kdims, kstr, box) || !make_tmap(&to, o, 3, qdims, qstr, box))
+    return FRT_ERR_CUDA;
+  PrefillParams p;
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.g = Hq / Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.causal = causal;
+  p.n_qtiles = n_qtiles;
+  p.scale_log2 = scale * kLog2e;
+  const dim3 grid((unsigned)(B * Hq), (unsigned)n_qtiles);
+  if (D == 128)
+    prefill_kernel<128><<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
+  else
+    prefill_kernel<64><<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace frt
+
+using namespace frt;
+
+extern "C" {
+
+frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, int max_pages_per_seq,
+                                 const int32_t* seq_lens, int page_size, int num_pages,
+                                 void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                 float scale, int num_splits, void* workspace,
+                                 size_t* workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq < 0 ||
+      num_splits < 0 || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
+  if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  if (q != nullptr && B > 0) {
+    if (k_pages == nullptr || v_pages == nullptr || o == nullptr ||
+        seq_lens == nullptr || (block_table == nullptr && max_pages_per_seq > 0))
+      return FRT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
+        (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+      return FRT_ERR_INVALID_ARG;
+    if (num_pages == 0) return FRT_ERR_INVALID_ARG;
+  }
+  return launch_decode(q, k_pages, v_pages, (uint64_t)num_pages * Hkv * page_size, block_table,
+                       max_pages_per_seq, seq_lens, 0, o, lse, B, Hq, Hkv, D, scale,
+                       num_splits, workspace, workspace_bytes, stream);
+}
+
+frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Sq, int Skv, int D, int causal, float scale,
+                        void* workspace, size_t* workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Skv < 0 ||
+      (causal != 0 && causal != 1) || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)B * Hkv * Skv >= (1ull << 31) || (uint64_t)B * Hq * Sq >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
+  const bool decode = (Sq == 1 && Skv > 0);
+  if (q == nullptr) {   // size query
+    if (workspace_bytes == nullptr) return FRT_ERR_INVALID_ARG;
+    if (!decode) {
+      *workspace_bytes = 0;
+      return FRT_OK;
+    }
+    return launch_decode(nullptr, k, v, (uint64_t)B * Hkv * Skv, nullptr, 0, nullptr, Skv, o,
+                         lse, B, Hq, Hkv, D, scale, 0, nullptr, workspace_bytes, stream);
+  }
+  if (B == 0 || Sq == 0) return FRT_OK;
+  if (o == nullptr || (Skv > 0 && (k == nullptr || v == nullptr)))
+    return FRT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FRT_ERR_INVALID_ARG;
+  if (decode) {
+    if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
+    return launch_decode(q, k, v, (uint64_t)B * Hkv * Skv, nullptr, 0, nullptr, Skv, o, lse, B,
+                         Hq, Hkv, D, scale, 0, workspace, workspace_bytes, stream);
+  }
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream);
+}
+
+frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_parts, int S, int B,
+                              int Hq, int D, void* o, float* lse, cudaStream_t stream) {
+  if (S <= 0 || B < 0 || Hq <= 0) return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * Hq;
+  if (rows == 0) return FRT_OK;
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return FRT_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FRT_ERR_INVALID_ARG;
+  const long long blocks = (rows + kMergeWarps - 1) / kMergeWarps;
+  if (blocks > 0x7fffffffLL) return FRT_ERR_UNSUPPORTED;
+  if (D == 128)
+    merge_lse_kernel<128><<<(unsigned)blocks, kMergeWarps * 32, 0, stream>>>(
+        o_parts, lse_parts, S, rows, static_cast<__nv_bfloat16*>(o), lse);
+  else
+    merge_lse_kernel<64><<<(unsigned)blocks, kMergeWarps * 32, 0, stream>>>(
+        o_parts, lse_parts, S, rows, static_cast<__nv_bfloat16*>(o), lse);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+frt_status frt_read_device_error(unsigned* flags) {
+  if (flags == nullptr) return FRT_ERR_INVALID_ARG;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, frt_device_error, sizeof v) != cudaSuccess) return FRT_ERR_CUDA;
+  if (cudaMemcpyToSymbol(frt_device_error, &zero, sizeof zero) != cudaSuccess)
+    return FRT_ERR_CUDA;
+  *flags = v;
+  return FRT_OK;
+}
+
+const char* frt_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+"""Python binding of libfrt_attn.so (argument marshalling only).
+
+Every call hands raw device pointers, sizes and the current CUDA stream to
+the C ABI declared in include/frt_attn.h; all of the attention arithmetic
+runs in the library's CUDA kernels.  There is no fallback: if the library is
+missing or a call is rejected, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
+
+EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_merge_lse",
+           "frt_read_device_error", "frt_version")
+
+STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
+          3: "FRT_ERR_WORKSPACE", 4: "FRT_ERR_CUDA"}
+
+
+class FrtError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m flash_attention_tiled_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_size_t)
+    lib.frt_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
+    lib.frt_attn_decode_paged.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I, P, Z, P]
+    lib.frt_attn_merge_lse.argtypes = [P, P, I, I, I, I, P, P, P]
+    lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    for name in EXPORTS[:-1]:
+        getattr(lib, name).restype = ctypes.c_int
+    lib.frt_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def version() -> str:
+    return _lib.frt_version().decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise FrtError(fn, rc)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# Zero-filled workspaces, one per (device, stream, shape): the library's
+# arrival counters return to zero after every call, so a workspace can be
+# reused by later calls of the same shape ordered on the same stream.
+_workspaces: dict = {}
+
+
+def workspace(nbytes: int, device, stream_handle: int, shape_key=()) -> torch.Tensor:
+    key = (torch.device(device).index, stream_handle, nbytes, shape_key)
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, return_lse: bool = True):
+    """o, lse = attention(q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D]) with bf16 tensors."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 4)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    stream = _stream(q.device)
+    need = ctypes.c_size_t(0)
+    _check("frt_attn_fwd", _lib.frt_attn_fwd(None, None, None, None, None, B, Hq, Hkv, Sq, Skv,
+                                             D, int(causal), scale, None, ctypes.byref(need),
+                                             stream))
+    ws = None
+    if need.value > 0:
+        ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, 0))
+        need = ctypes.c_size_t(ws.numel())
+    _check("frt_attn_fwd", _lib.frt_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
+                                             Hq, Hkv, Sq, Skv, D, int(causal), scale, _ptr(ws),
+                                             ctypes.byref(need), stream))
+    return out, lse
+
+
+def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                      block_table: torch.Tensor, seq_lens: torch.Tensor,
+                      scale: float | None = None, num_splits: int = 0,
+                      out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                      return_lse: bool = True):
+    """o, lse = decode attention of q [B,Hq,D] over pages [P,Hkv,ps,D] (bf16)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    stream = _stream(q.device)
+    need = ctypes.c_size_t(0)
+    _check("frt_attn_decode_paged", _lib.frt_attn_decode_paged(
+        None, None, None, None, block_table.shape[1], None, ps, P, None, None, B, Hq, Hkv, D,
+        scale, num_splits, None, ctypes.byref(need), stream))
+    ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, num_splits))
+    need = ctypes.c_size_t(ws.numel())
+    _check("frt_attn_decode_paged", _lib.frt_attn_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale, num_splits,
+        _ptr(ws), ctypes.byref(need), stream))
+    return out, lse
+
+
+def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor | None = None,
+              lse: torch.Tensor | None = None, return_lse: bool = True):
+    """o [B,Hq,D] bf16, lse [B,Hq] = merge of o_parts [S,B,Hq,D], lse_parts [S,B,Hq] (fp32)."""
+    _need(o_parts, "o_parts", torch.float32, 4)
+    _need(lse_parts, "lse_parts", torch.float32, 3)
+    S, B, Hq, D = o_parts.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=o_parts.device)
+    _check("frt_attn_merge_lse", _lib.frt_attn_merge_lse(
+        _ptr(o_parts), _ptr(lse_parts), S, B, Hq, D, _ptr(out), _ptr(lse),
+        _stream(o_parts.device)))
+    return out, lse
+
+
+def read_device_error() -> int:
+    """Read and clear the library's device-side error word (synchronises)."""
+    flags = ctypes.c_uint(0)
+    _check("frt_read_device_error", _lib.frt_read_device_error(ctypes.byref(flags)))
+    return flags.value

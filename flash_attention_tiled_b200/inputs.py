@@ -127,10 +127,11 @@ def make(workload: Workload | str) -> dict:
 
 def partials(S, rows, D, seed, empty_frac=0.0) -> dict:
     """Random partial results for the log-sum-exp merge: o_parts [S,rows,D] fp32
-    ~ N(0,1), lse_parts [S,rows] fp32 ~ N(0, 4); a fraction of the parts is
-    marked empty (lse = -inf)."""
+    ~ N(0, 1/4) (a partial attention output is a convex combination of value
+    rows, so it is smaller than one value row), lse_parts [S,rows] fp32
+    ~ N(0, 4); a fraction of the parts is marked empty (lse = -inf)."""
     gen = torch.Generator("cpu").manual_seed(seed)
-    o_parts = torch.randn((S, rows, D), generator=gen, dtype=torch.float32)
+    o_parts = 0.5 * torch.randn((S, rows, D), generator=gen, dtype=torch.float32)
     lse_parts = 2.0 * torch.randn((S, rows), generator=gen, dtype=torch.float32)
     if empty_frac > 0:
         drop = torch.rand((S, rows), generator=gen) < empty_frac

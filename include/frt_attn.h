@@ -1,0 +1,174 @@
+/*
+ * frt_attn.h -- C ABI of the B200 (sm_100a) fused-attention library.
+ *
+ * Three operations, each the FlashAttention-style computation of softmax
+ * attention that the pages describe:
+ *   - "Real-time inference optimisation: making large models respond fast"
+ *     (llmapi-app.pages.dev), section "Flash Attention optimisation": tiled
+ *     Q.K^T times a scale, online softmax (running max and sum, rescaling the
+ *     accumulator), P.V accumulation, final division by the sum; method
+ *     paged_attention: a KV cache in pages of 16 tokens.
+ *   - "FlashRT-HF-kernels" (zingnex.cn), section "Attention optimisation":
+ *     blockwise computation without storing the attention matrix, causal
+ *     masking for autoregressive generation, MQA/GQA; section "Attention
+ *     operators": flash attention, cross attention, paged attention.
+ *   - "Analysis of TensorRT's low-level support for FlashAttention"
+ *     (yongjin360.com), the plugin
+ *     sketch: the kernel is launched on the caller's stream with Q, K, V, O,
+ *     head count, query and key lengths and head dimension, and returns 0.
+ *
+ * Definition computed (all three calls).  For batch b, query head h, query i,
+ * with g = Hq / Hkv and KV head kvh = h / g:
+ *   s_ij = scale * sum_d q[b,h,i,d] * k[b,kvh,j,d]
+ *   key j is visible to query i iff  !causal || j <= i + (Skv - Sq)
+ *   o[b,h,i,:] = sum_j softmax_j(s_ij) * v[b,kvh,j,:]   over visible j
+ *   lse[b,h,i] = log(sum_j exp(s_ij))                    natural log, scale included
+ * A row with no visible key gets o = 0 and lse = -inf.  The causal mask is
+ * aligned bottom-right (the last query sees every key), which is the usual
+ * lower-triangular mask when Sq == Skv; the pages do not fix the alignment
+ * for Sq != Skv, this is the library's reading.
+ *
+ * Conventions shared by every call:
+ *   - All pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or synchronises.  Every call is asynchronous on
+ *     `stream`; a device-side failure (an internal wait that timed out) is
+ *     reported by frt_read_device_error(), never by a hang.
+ *   - Tensors are contiguous, row-major, with the shapes given; q/k/v/o are
+ *     bf16 (uint16 bit patterns), lse is fp32.  Every pointer must be 16-byte
+ *     aligned.  Head dimension D is 64 or 128.
+ *   - Arguments are validated before anything is launched; a rejected call
+ *     returns a non-zero status and leaves every output untouched.
+ *   - Arithmetic: bf16 inputs, fp32 accumulation, exp2-based softmax with
+ *     the scale folded into the exponent, P rounded to bf16 before the P.V
+ *     product, O rounded once to bf16 (round to nearest even).
+ */
+#ifndef FRT_ATTN_H_
+#define FRT_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FRT_API __attribute__((visibility("default")))
+#else
+#define FRT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FRT_OK = 0,
+  FRT_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, Hq % Hkv != 0, bad scale */
+  FRT_ERR_UNSUPPORTED = 2,   /* valid but not implemented here (e.g. D not in {64,128}) */
+  FRT_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  FRT_ERR_CUDA = 4           /* a CUDA runtime call failed (launch, attribute query) */
+} frt_status;
+
+/*
+ * frt_attn_fwd -- attention over a contiguous KV tensor (prefill, chunked
+ * prefill, cross attention and single-token decode).
+ *
+ *   q   [B, Hq,  Sq,  D] bf16      k, v  [B, Hkv, Skv, D] bf16
+ *   o   [B, Hq,  Sq,  D] bf16      lse   [B, Hq, Sq] fp32, may be NULL
+ *   causal: 0 or 1 (bottom-right aligned, see above); scale > 0 and finite
+ *   (1/sqrt(D) in the usual model).
+ *
+ * Sq > 1 runs the tiled tensor-core kernel (128-query tiles, 128-key tiles,
+ * fully masked key tiles skipped).  Sq == 1 runs the split-KV decode kernel
+ * over the contiguous cache; that path needs a workspace like
+ * frt_attn_decode_paged (same rules) and takes it from `workspace`.
+ * Size query: a call with q == NULL only writes the workspace size to
+ * *workspace_bytes (0 when Sq > 1) and returns FRT_OK; workspace and
+ * workspace_bytes may be NULL on real calls that need none (Sq > 1).
+ * B, Sq or Skv may be 0 (nothing to attend: o = 0, lse = -inf where rows
+ * exist).
+ */
+FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
+                        float scale, void* workspace, size_t* workspace_bytes,
+                        cudaStream_t stream);
+
+/*
+ * frt_attn_decode_paged -- one query token per sequence over a paged KV
+ * cache ("Real-time inference optimisation" page, method paged_attention:
+ * pages of 16 tokens; "FlashRT-HF-kernels" page, "Attention operators":
+ * paged attention).
+ *
+ *   q           [B, Hq, D] bf16
+ *   k_pages,
+ *   v_pages     [num_pages, Hkv, page_size, D] bf16: physical pages; each
+ *               (page, KV head) is one contiguous page_size x D block
+ *   block_table [B, max_pages_per_seq] int32: token t of sequence b is in
+ *               physical page block_table[b][t / page_size], slot
+ *               t % page_size; entries past a sequence's last page are
+ *               never read
+ *   seq_lens    [B] int32 on the device: tokens in each sequence; a value
+ *               above max_pages_per_seq * page_size is clamped to it, a
+ *               negative one is read as 0
+ *   o           [B, Hq, D] bf16;  lse [B, Hq] fp32, may be NULL
+ *   page_size   16 in this version
+ *   num_splits  number of work partitions the cache is cut into (0 = one
+ *               per SM, the default); every partition streams an equal
+ *               share of all sequences' pages, so mixed lengths balance
+ *   workspace   device scratch of *workspace_bytes bytes, 16-byte aligned.
+ *               Size query: a call with q == NULL only writes the required
+ *               size to *workspace_bytes and returns FRT_OK.  The size
+ *               depends on B, Hq, Hkv, D and num_splits only.  It holds
+ *               arrival counters that must read zero when a call starts:
+ *               zero-fill a workspace before its first use; every call
+ *               leaves the counters at zero again, so later calls with the
+ *               same shape may reuse it as is.  A workspace last used for a
+ *               different shape (or a call that reported a device error)
+ *               must be zero-filled again first.  Calls that share a
+ *               workspace must be ordered on the device (the same stream,
+ *               or events).
+ *
+ * Block-table entries outside [0, num_pages) read zeros (the copy engine's
+ * bounds), never out-of-bounds memory.  Tail slots of the last page of a
+ * sequence may hold anything, NaN included: they never reach o.
+ */
+FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, int max_pages_per_seq,
+                                 const int32_t* seq_lens, int page_size, int num_pages,
+                                 void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                 float scale, int num_splits, void* workspace,
+                                 size_t* workspace_bytes, cudaStream_t stream);
+
+/*
+ * frt_attn_merge_lse -- combine S partial attention results of the same rows,
+ * each computed over a disjoint set of keys, into the result over their
+ * union.  This is the correct form of the per-page combination in the
+ * "Real-time inference optimisation" page's paged_attention method (which
+ * adds normalised per-page outputs): with lse = log sum_s exp(lse_s),
+ *   o = sum_s exp(lse_s - lse) * o_s.
+ * It is the same algebra as the online-softmax update of that page's
+ * "Flash Attention optimisation" section.
+ *
+ *   o_parts   [S, rows, D] fp32 (rows = B * Hq), each normalised
+ *   lse_parts [S, rows] fp32 natural-log LSE; -inf marks an empty part
+ *   o         [rows, D] bf16;  lse [rows] fp32, may be NULL
+ * A row whose parts are all empty gets o = 0, lse = -inf.  S >= 1.
+ */
+FRT_API frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_parts, int S, int B,
+                              int Hq, int D, void* o, float* lse, cudaStream_t stream);
+
+/*
+ * frt_read_device_error -- read and clear the library's device-side error
+ * word on the current device (synchronises that device).  0 means no kernel
+ * gave up; bit 0 = an internal wait timed out (the kernel returned without
+ * finishing its outputs).  Returns FRT_ERR_CUDA if the read itself failed.
+ */
+FRT_API frt_status frt_read_device_error(unsigned* flags);
+
+/* Library version string ("major.minor.patch"). */
+FRT_API const char* frt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FRT_ATTN_H_ */

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+call that include/*.h declares, and rejects bad arguments before touching
+the device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from flash_attention_tiled_b200 import frt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"FRT_API\s+[\w\s\*]*?\b(frt_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared()
+    assert set(frt.EXPORTS) <= set(declared)
+    for name in declared:
+        assert hasattr(frt.lib(), name), name     # ctypes resolves it with dlsym
+
+
+def test_version():
+    assert re.fullmatch(r"\d+\.\d+\.\d+", frt.version())
+
+
+NULL = None
+Z = ctypes.c_size_t
+
+
+def _fwd(B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64, causal=0, scale=0.125, query=True):
+    need = Z(0)
+    return frt.lib().frt_attn_fwd(NULL, NULL, NULL, NULL, NULL, B, Hq, Hkv, Sq, Skv, D, causal,
+                                  scale, NULL, ctypes.byref(need), NULL), need.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), 1),               # Hq % Hkv != 0
+    (dict(Hkv=0), 1),
+    (dict(B=-1), 1),
+    (dict(Sq=-2), 1),
+    (dict(causal=2), 1),
+    (dict(scale=0.0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1),
+    (dict(D=96), 2),                      # head dim not built
+    (dict(D=256), 2),
+])
+def test_fwd_rejects(kw, code):
+    rc, _ = _fwd(**kw)
+    assert rc == code
+
+
+def test_fwd_prefill_needs_no_workspace():
+    rc, need = _fwd(Sq=64, Skv=64)
+    assert rc == 0 and need == 0
+
+
+def _paged(B=1, Hq=8, Hkv=2, D=128, ps=16, num_pages=4, maxp=2, splits=0, scale=0.1):
+    need = Z(0)
+    return frt.lib().frt_attn_decode_paged(NULL, NULL, NULL, NULL, maxp, NULL, ps, num_pages,
+                                           NULL, NULL, B, Hq, Hkv, D, scale, splits, NULL,
+                                           ctypes.byref(need), NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=6, Hkv=4), 1), (dict(scale=-1.0), 1), (dict(splits=-1), 1), (dict(num_pages=-1), 1),
+    (dict(maxp=-1), 1), (dict(D=80), 2), (dict(ps=8), 2), (dict(ps=32), 2), (dict(B=5000), 2),
+])
+def test_decode_rejects(kw, code):
+    assert _paged(**kw) == code
+
+
+def test_decode_workspace_query_with_explicit_splits():
+    # with an explicit split count the size needs no device query
+    need = Z(0)
+    rc = frt.lib().frt_attn_decode_paged(NULL, NULL, NULL, NULL, 8, NULL, 16, 10, NULL, NULL, 2,
+                                         64, 8, 128, 0.1, 37, NULL, ctypes.byref(need), NULL)
+    assert rc == 0
+    # partials for 37 + 16 slots of 16 rows x 128 fp32, LSEs and 16 counters
+    assert need.value >= (37 + 16) * 16 * 128 * 4 + (37 + 16) * 16 * 4 + 16 * 4
+
+
+@pytest.mark.parametrize("S,B,Hq,D,code", [(0, 1, 1, 64, 1), (1, -1, 1, 64, 1), (2, 1, 0, 64, 1),
+                                           (2, 1, 1, 32, 2)])
+def test_merge_rejects(S, B, Hq, D, code):
+    assert frt.lib().frt_attn_merge_lse(NULL, NULL, S, B, Hq, D, NULL, NULL, NULL) == code
+
+
+def test_merge_empty_rows_is_a_noop():
+    assert frt.lib().frt_attn_merge_lse(NULL, NULL, 3, 0, 4, 64, NULL, NULL, NULL) == 0

@@ -1,0 +1,287 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Bar (all outputs are bf16 from fp32 accumulation): max |o - o_ref| <= 1e-2,
+mean |o - o_ref| <= 1e-3, max |lse - lse_ref| <= 1e-3; index work (which
+page, which slot) bit-exact.  The five named workloads run at full size;
+where the oracle would take too long (the 4k prefill) it checks sampled rows,
+computed one by one, of the very launch the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from flash_attention_tiled_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS, LSE_ABS = 1e-2, 1e-3, 1e-3
+
+
+@pytest.fixture(scope="module")
+def frt():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from flash_attention_tiled_b200 import frt as f
+    return f
+
+
+def _compare(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
+    o = o_gpu.detach().float().cpu().double().numpy().reshape(o_ref.shape)
+    assert np.isfinite(o).all(), f"{what}: non-finite output"
+    err = np.abs(o - o_ref)
+    assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3g}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean abs err {err.mean():.3g}"
+    if lse_gpu is not None:
+        lg = lse_gpu.detach().cpu().double().numpy().reshape(lse_ref.shape)
+        fin = np.isfinite(lse_ref)
+        assert np.array_equal(np.isneginf(lg), np.isneginf(lse_ref)), f"{what}: -inf rows differ"
+        if fin.any():
+            lerr = np.abs(lg[fin] - lse_ref[fin])
+            assert lerr.max() <= LSE_ABS, f"{what}: lse err {lerr.max():.3g}"
+    return err.max()
+
+
+def _dev(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def _no_device_error(frt):
+    assert frt.read_device_error() == 0
+
+
+# ------------------------------------------------------------ named workloads
+def test_tiny_causal(frt):
+    w = inputs.WORKLOADS["tiny_causal"]
+    x = inputs.make(w)
+    d = _dev(x)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], True, w.scale)
+    _compare(o, o_ref, lse, lse_ref, "tiny_causal")
+    # causal row 0 attends to key 0 alone: p = 1 exactly, so o = v[0] bit-exactly
+    assert torch.equal(o[:, :, 0].cpu(), x["v"][:, :, 0])
+    _no_device_error(frt)
+
+
+def test_gqa_decode_contiguous(frt):
+    w = inputs.WORKLOADS["gqa_decode_4k"]
+    x = inputs.make(w)
+    d = _dev(x)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=False, scale=w.scale)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], False, w.scale)
+    _compare(o, o_ref, lse, lse_ref, "gqa_decode_4k")
+    _no_device_error(frt)
+
+
+def test_llama3_prefill_sampled_rows(frt):
+    w = inputs.WORKLOADS["llama3_8b_prefill_4k"]
+    x = inputs.make(w)
+    d = _dev(x)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    gen = np.random.default_rng(7)
+    rows = []
+    for h in (0, 5, 17, 31):
+        base = h * w.Sq
+        rows += [base + i for i in (0, 1, 2, 3, 127, 128, 129, 255, 1000, 2047, 2048, 4094, 4095)]
+    rows += list(gen.integers(0, w.Hq * w.Sq, size=200))
+    rows = np.array(sorted(set(int(r) for r in rows)), dtype=np.int64)
+    o_ref, lse_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], True, w.scale, rows)
+    _compare(o.reshape(-1, w.D)[torch.from_numpy(rows).cuda()], o_ref,
+             lse.reshape(-1)[torch.from_numpy(rows).cuda()], lse_ref, "prefill sampled")
+    # properties that hold at any size: row 0 of every head is v[0] exactly,
+    # and every output lies in the convex hull of the values it attends
+    kvh = torch.arange(w.Hq, device="cuda") // (w.Hq // w.Hkv)
+    assert torch.equal(o[0, :, 0], d["v"][0, kvh, 0])
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    vmax = d["v"].float().abs().amax().item()
+    assert o.float().abs().amax().item() <= vmax
+    _no_device_error(frt)
+
+
+def _paged_case(frt, x, scale, num_splits=0, what=""):
+    d = _dev(x)
+    o, lse = frt.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
+                                   d["seq_lens"], scale=scale, num_splits=num_splits)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_decode_paged(x["q"], x["k_pages"], x["v_pages"],
+                                              x["block_table"], x["seq_lens"], scale)
+    _compare(o, o_ref, lse, lse_ref, what)
+    return o, lse
+
+
+def test_paged_gqa_decode(frt):
+    w = inputs.WORKLOADS["paged_gqa_decode_b4"]
+    _paged_case(frt, inputs.make(w), w.scale, what=w.name)
+    _no_device_error(frt)
+
+
+def test_long_splitkv_decode(frt):
+    w = inputs.WORKLOADS["long_splitkv_decode_256k"]
+    _paged_case(frt, inputs.make(w), w.scale, what=w.name)
+    _no_device_error(frt)
+
+
+# --------------------------------------------------------- prefill edge cases
+PREFILL_CASES = [  # B, Hq, Hkv, Sq, Skv, D, causal
+    (1, 2, 2, 128, 128, 64, False),
+    (2, 4, 2, 200, 200, 128, True),     # ragged tail, GQA
+    (1, 4, 1, 77, 333, 128, True),      # MQA, Sq < Skv (bottom-right)
+    (1, 2, 2, 333, 77, 64, True),       # Sq > Skv: leading rows see no key
+    (1, 2, 1, 256, 1000, 128, False),   # cross attention shape
+    (2, 2, 2, 129, 129, 64, True),
+    (1, 1, 1, 2, 1, 128, False),        # Skv = 1: o = v
+    (1, 2, 2, 513, 513, 128, True),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=str)
+def test_prefill_edge(frt, case):
+    B, Hq, Hkv, Sq, Skv, D, causal = case
+    x = inputs.dense(B, Hq, Hkv, Sq, Skv, D, seed=sum(case) + 17)
+    d = _dev(x)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], causal, scale)
+    _compare(o, o_ref, lse, lse_ref, str(case))
+    _no_device_error(frt)
+
+
+def test_prefill_large_scores_rescale(frt):
+    # scores spread over hundreds of log2 units force the lazy rescale path
+    x = inputs.dense(1, 2, 2, 300, 300, 128, seed=5)
+    x["q"] = (x["q"].float() * 6).to(torch.bfloat16)
+    d = _dev(x)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=0.5)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], True, 0.5)
+    _compare(o, o_ref, lse, lse_ref, "large scores")
+
+
+def test_prefill_empty_keys(frt):
+    x = inputs.dense(1, 2, 2, 5, 1, 64, seed=3)
+    d = _dev(x)
+    k0 = d["k"][:, :, :0].contiguous()
+    v0 = d["v"][:, :, :0].contiguous()
+    o = torch.full_like(d["q"], 7.0)
+    o, lse = frt.attn_fwd(d["q"], k0, v0, causal=False, out=o)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_prefill_deterministic(frt):
+    x = _dev(inputs.dense(1, 4, 2, 384, 384, 128, seed=9))
+    o1, l1 = frt.attn_fwd(x["q"], x["k"], x["v"], causal=True)
+    o2, l2 = frt.attn_fwd(x["q"], x["k"], x["v"], causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------- decode edge cases
+DECODE_CASES = [  # lens, Hq, Hkv, D, num_splits
+    ([1], 8, 8, 128, 0),
+    ([15, 16, 17, 33], 8, 2, 128, 0),
+    ([5000, 0, 300], 32, 4, 128, 0),      # an empty sequence
+    ([4096], 32, 1, 128, 0),              # MQA, two head groups of 16
+    ([1000, 2000], 16, 16, 64, 0),        # g = 1, D = 64
+    ([3333, 77], 24, 2, 128, 1),          # one partition: no merge
+    ([3333, 77], 24, 2, 128, 3),
+    ([3333, 77], 24, 2, 128, 1000),       # more partitions than pages
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=str)
+def test_decode_edge(frt, case):
+    lens, Hq, Hkv, D, splits = case
+    x = inputs.paged(len(lens), Hq, Hkv, D, seq_lens=lens, seed=len(lens) * 31 + Hq)
+    o, lse = _paged_case(frt, x, 1.0 / math.sqrt(D), splits, str(case))
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
+    _no_device_error(frt)
+
+
+def test_decode_contiguous_ragged(frt):
+    for Skv in (1, 7, 16, 100, 1025):
+        x = inputs.dense(2, 8, 2, 1, Skv, 128, seed=Skv)
+        d = _dev(x)
+        o, lse = frt.attn_fwd(d["q"], d["k"], d["v"])
+        torch.cuda.synchronize()
+        o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], False, 1 / math.sqrt(128))
+        _compare(o, o_ref, lse, lse_ref, f"contiguous decode Skv={Skv}")
+
+
+@pytest.mark.parametrize("t_star", [0, 15, 16, 17, 4095, 4096, 4099])
+def test_decode_page_indexing_probe(frt, t_star):
+    # all keys 0 except logical token t*, whose key makes p one-hot: the output
+    # must be that token's value row bit-exactly (wrong page or slot -> wrong row)
+    B, Hq, Hkv, D, n = 2, 8, 2, 128, 4100
+    x = inputs.paged(B, Hq, Hkv, D, seq_lens=[n, n - 37], seed=t_star)
+    q = torch.zeros_like(x["q"])
+    q[:, :, 0] = 1.0
+    kp = torch.zeros_like(x["k_pages"])
+    for b in range(B):
+        if t_star < int(x["seq_lens"][b]):
+            phys = int(x["block_table"][b, t_star // 16])
+            kp[phys, :, t_star % 16, 0] = 256.0   # score 256*scale' >> others
+    x["q"], x["k_pages"] = q, kp
+    d = _dev(x)
+    o, _ = frt.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
+                                 d["seq_lens"], scale=1.0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        if t_star >= int(x["seq_lens"][b]):
+            continue
+        phys = int(x["block_table"][b, t_star // 16])
+        for h in range(Hq):
+            assert torch.equal(o[b, h].cpu(), x["v_pages"][phys, h // (Hq // Hkv), t_star % 16])
+
+
+def test_decode_deterministic(frt):
+    x = _dev(inputs.paged(3, 16, 2, 128, seq_lens=[9000, 100, 20000], seed=4))
+    args = (x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"])
+    o1, l1 = frt.attn_decode_paged(*args)
+    o2, l2 = frt.attn_decode_paged(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_decode_splits_agree(frt):
+    # any partition of the keys merges to the same result (within fp32 rounding;
+    # the LSE goes through the approximate exp2/log2 units, ~1e-5 relative)
+    x = _dev(inputs.paged(2, 16, 2, 128, seq_lens=[7000, 3001], seed=8))
+    args = (x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"])
+    o1, l1 = frt.attn_decode_paged(*args, num_splits=1)
+    for s in (2, 7, 148, 600):
+        o2, l2 = frt.attn_decode_paged(*args, num_splits=s)
+        torch.cuda.synchronize()
+        assert (o1.float() - o2.float()).abs().max().item() <= 2 ** -7
+        assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+# ------------------------------------------------------------------- merge
+@pytest.mark.parametrize("S,B,Hq,D,empty", [(1, 2, 8, 128, 0.0), (5, 3, 16, 128, 0.3),
+                                            (37, 1, 32, 128, 0.0), (4, 2, 4, 64, 0.5)])
+def test_merge_lse(frt, S, B, Hq, D, empty):
+    x = inputs.partials(S, B * Hq, D, seed=S * 100 + D, empty_frac=empty)
+    op = x["o_parts"].reshape(S, B, Hq, D)
+    lp = x["lse_parts"].reshape(S, B, Hq)
+    o, lse = frt.merge_lse(op.cuda(), lp.cuda())
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.merge_lse(op.numpy(), lp.numpy())
+    _compare(o, o_ref, lse, lse_ref, "merge")
+    if S == 1:
+        assert torch.equal(o.cpu(), op[0].to(torch.bfloat16))
+
+
+def test_merge_all_empty_row(frt):
+    op = torch.randn(3, 1, 2, 64)
+    lp = torch.full((3, 1, 2), -math.inf)
+    o, lse = frt.merge_lse(op.cuda(), lp.cuda())
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
