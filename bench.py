@@ -146,36 +146,32 @@ class ClockSampler:
 class Step:
     """The four calls of one step, with inputs resident on the device."""
 
-    def __init__(self, device):
+    ALL = ("prefill", "paged", "long", "contig")
+
+    def __init__(self, device, names=ALL):
         from flash_attention_tiled_b200 import frt
         self.frt = frt
         self.dev = device
+        self.NAMES = tuple(names)
         W = inputs.WORKLOADS
         self.w_pf = W["llama3_8b_prefill_4k"]
         self.w_pg = W["paged_gqa_decode_b4"]
         self.w_lg = W["long_splitkv_decode_256k"]
         self.w_ct = W["gqa_decode_4k"]
-        self.host = {
-            "prefill": inputs.make(self.w_pf),
-            "paged": inputs.make(self.w_pg),
-            "long": inputs.make(self.w_lg),
-            "contig": inputs.make(self.w_ct),
-        }
+        wl = {"prefill": self.w_pf, "paged": self.w_pg, "long": self.w_lg, "contig": self.w_ct}
+        self.host = {n: inputs.make(wl[n]) for n in self.NAMES}
         self.d = {k: {n: (t.to(device) if isinstance(t, torch.Tensor) else t)
                       for n, t in v.items()} for k, v in self.host.items()}
-        self.tokens_pg = int(self.host["paged"]["seq_lens"].sum())
-        self.tokens_lg = int(self.host["long"]["seq_lens"].sum())
+        if "paged" in self.NAMES:
+            self.tokens_pg = int(self.host["paged"]["seq_lens"].sum())
+        if "long" in self.NAMES:
+            self.tokens_lg = int(self.host["long"]["seq_lens"].sum())
         # outputs, allocated once
-        self.out = {
-            "prefill": (torch.empty_like(self.d["prefill"]["q"]),
-                        torch.empty(self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq, device=device)),
-            "paged": (torch.empty_like(self.d["paged"]["q"]),
-                      torch.empty(self.w_pg.B, self.w_pg.Hq, device=device)),
-            "long": (torch.empty_like(self.d["long"]["q"]),
-                     torch.empty(self.w_lg.B, self.w_lg.Hq, device=device)),
-            "contig": (torch.empty_like(self.d["contig"]["q"]),
-                       torch.empty(self.w_ct.B, self.w_ct.Hq, 1, device=device)),
-        }
+        shapes = {"prefill": (self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq),
+                  "paged": (self.w_pg.B, self.w_pg.Hq), "long": (self.w_lg.B, self.w_lg.Hq),
+                  "contig": (self.w_ct.B, self.w_ct.Hq, 1)}
+        self.out = {n: (torch.empty_like(self.d[n]["q"]), torch.empty(shapes[n], device=device))
+                    for n in self.NAMES}
 
     def call(self, name, d=None, out=None):
         d = self.d[name] if d is None else d
@@ -190,66 +186,98 @@ class Step:
             f.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
                                 d["seq_lens"], scale=w.scale, out=o, lse=l)
 
-    NAMES = ("prefill", "paged", "long", "contig")
-
     def work(self):
         """Algorithmic (flops, bytes) of each call."""
-        pf = self.w_pf
-        return {
-            "prefill": (prefill_flops(pf), prefill_bytes(pf)),
-            "paged": (decode_flops(self.w_pg.Hq, 128, self.tokens_pg),
-                      decode_bytes(self.w_pg.B, self.w_pg.Hq, self.w_pg.Hkv, 128, self.tokens_pg)),
-            "long": (decode_flops(self.w_lg.Hq, 128, self.tokens_lg),
-                     decode_bytes(1, self.w_lg.Hq, self.w_lg.Hkv, 128, self.tokens_lg)),
-            "contig": (decode_flops(self.w_ct.Hq, 128, self.w_ct.Skv),
-                       decode_bytes(1, self.w_ct.Hq, self.w_ct.Hkv, 128, self.w_ct.Skv)),
-        }
+        out = {}
+        for n in self.NAMES:
+            if n == "prefill":
+                out[n] = (prefill_flops(self.w_pf), prefill_bytes(self.w_pf))
+            elif n == "paged":
+                out[n] = (decode_flops(self.w_pg.Hq, 128, self.tokens_pg),
+                          decode_bytes(self.w_pg.B, self.w_pg.Hq, self.w_pg.Hkv, 128,
+                                       self.tokens_pg))
+            elif n == "long":
+                out[n] = (decode_flops(self.w_lg.Hq, 128, self.tokens_lg),
+                          decode_bytes(1, self.w_lg.Hq, self.w_lg.Hkv, 128, self.tokens_lg))
+            else:
+                out[n] = (decode_flops(self.w_ct.Hq, 128, self.w_ct.Skv),
+                          decode_bytes(1, self.w_ct.Hq, self.w_ct.Hkv, 128, self.w_ct.Skv))
+        return out
 
 
 def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    st = Step(device)
-    stream = torch.cuda.current_stream(device)
-    names = Step.NAMES
-    for _ in range(args.warmup):
+    st = Step(device, args.calls)
+    names = st.NAMES
+    # Everything runs on one dedicated stream; the step and each call are
+    # captured once as CUDA graphs, so the device time measured is the
+    # kernels' and not the host's launch overhead.
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for n in names:
+                st.call(n)
+    torch.cuda.synchronize(device)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
         for n in names:
             st.call(n)
+    g_call = {}
+    for n in names:
+        g_call[n] = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_call[n], stream=stream):
+            st.call(n)
+    # L2 flush for the per-call timings: write twice the L2 size
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_step.replay()
     torch.cuda.synchronize(device)
 
-    # per-call events over the whole timed region
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-          for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     sampler = ClockSampler(device.index if device.index is not None else 0)
-    with sampler:
+    with sampler, torch.cuda.stream(stream):
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         start.record(stream)
-        for s in range(args.steps):
-            e = ev[s]
-            e[0].record(stream)
-            for i, n in enumerate(names):
-                st.call(n)
-                e[i + 1].record(stream)
+        for _ in range(args.steps):
+            g_step.replay()
         end.record(stream)
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     total_ms = start.elapsed_time(end)
-    per_call_ms = {n: float(np.mean([ev[s][i].elapsed_time(ev[s][i + 1])
-                                     for s in range(args.steps)]))
-                   for i, n in enumerate(names)}
     if world > 1:
         t = torch.tensor([total_ms], device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
 
+    # per-call device time, each call starting with a flushed L2
+    reps = max(3, min(args.steps, 50))
+    per_call_ms = {}
+    with torch.cuda.stream(stream):
+        for n in names:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            for a, b in evs:
+                flush.fill_(1.0)
+                a.record(stream)
+                g_call[n].replay()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+            per_call_ms[n] = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(st, args, device)
+    e2e = None
+    if not args.no_e2e:
+        with torch.cuda.stream(stream):
+            e2e = run_e2e(st, args, device)
+    del g_step, g_call
 
     if rank != 0:
         return None
@@ -260,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
         fl, by = work[n]
         us = per_call_ms[n] * 1e3
         rec = {"us": round(us, 2), "tflops": round(fl / us * 1e-6, 1),
-               "gbs": round(by / us * 1e-3, 1)}
+               "gbs": round(by / us * 1e-3, 1), "flop": fl, "bytes": by}
         if n == "prefill":
             rec["bound"] = "tensor"
             rec["frac"] = round(rec["tflops"] / peaks["bf16_tflops"], 4)
@@ -268,19 +296,34 @@ def run_ours(args, rank, world, local_rank):
             rec["bound"] = "hbm"
             rec["frac"] = round(rec["gbs"] / peaks["hbm_gbs"], 4)
         calls[n] = rec
-    dom = max(names, key=lambda n: per_call_ms[n])
-    d = calls[dom]
-    if d["bound"] == "tensor":
-        roof = {"bound": "tensor", "achieved": d["tflops"], "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
+    # The dominant kernel is the one with the largest share of a step: the
+    # decode kernel serves three calls, the prefill kernel one.
+    kernel_of = {"prefill": "prefill_kernel<128>", "paged": "decode_splitkv_kernel<128>",
+                 "long": "decode_splitkv_kernel<128>", "contig": "decode_splitkv_kernel<128>"}
+    per_kernel = {}
+    for n in names:
+        k = kernel_of[n]
+        t, fl, by, cnt = per_kernel.get(k, (0.0, 0.0, 0.0, 0))
+        per_kernel[k] = (t + per_call_ms[n], fl + work[n][0], by + work[n][1], cnt + 1)
+    dom = max(per_kernel, key=lambda k: per_kernel[k][0])
+    t_ms, fl, by, cnt = per_kernel[dom]
+    if dom.startswith("prefill"):
+        roof = {"bound": "tensor", "achieved": round(fl / (t_ms * 1e-3) * 1e-12, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     else:
-        roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        roof = {"bound": "hbm", "achieved": round(by / (t_ms * 1e-3) * 1e-9, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["kernel"] = dom
+    roof["launches_per_step"] = cnt
+    roof["avg_launch_us"] = round(t_ms * 1e3 / cnt, 2)
     roof["peak_source"] = f"{peak_src} (burst figure: each kernel runs < 1 ms)"
     roof["traffic"] = None
+    roof["share_of_step"] = round(t_ms / sum(v[0] for v in per_kernel.values()), 3)
 
-    cpu = cpu_baseline(st, per_step_only=True)
+    cpu = None
+    if not args.no_cpu_baseline and tuple(names) == Step.ALL:
+        cpu = cpu_baseline(st)
     line = {
         "metric": METRIC,
         "value": round(world * args.steps / (total_ms * 1e-3), 2),
@@ -296,8 +339,11 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, shuffled page tables)",
         "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
                    "parallelism": f"replicas x{world}",
-                   "l2": "working set per step ~0.9 GB > 126 MB L2; each call's inputs are "
-                         "evicted by the calls before it (no explicit flush)"},
+                   "timing": "step = one CUDA graph of the four calls, replayed K times; "
+                             "per-call times: each call's own graph after an L2 flush",
+                   "l2": "step working set ~0.9 GB > 126 MB L2 and every call's inputs are "
+                         "evicted by the calls before it; per-call timings flush L2 "
+                         "(2x L2 size written) before each call"},
         "calls": calls,
         "roofline": roof,
         "cpu_baseline": cpu,
@@ -311,7 +357,7 @@ def run_ours(args, rank, world, local_rank):
 def run_e2e(st: Step, args, device):
     """Same step through the public API with pinned host inputs: H2D copy of
     every call's inputs, the call, and a D2H read of its outputs, per step."""
-    names = Step.NAMES
+    names = st.NAMES
     host = {n: {k: (t.pin_memory() if isinstance(t, torch.Tensor) else t)
                 for k, t in st.host[n].items()} for n in names}
     outs_h = {n: tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in st.out[n])
@@ -354,7 +400,7 @@ def cpu_sample_plan():
     return {"prefill_heads": 8, "paged_rows": 16, "long_heads": 4}
 
 
-def cpu_baseline(st: Step | None, per_step_only=False, host=None):
+def cpu_baseline(st: Step | None, host=None):
     import oracle
     plan = cpu_sample_plan()
     W = inputs.WORKLOADS
@@ -433,7 +479,15 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--calls", default=",".join(Step.ALL),
+                    help="comma-separated subset of the step's calls (profiling runs)")
     args = ap.parse_args()
+    args.calls = tuple(c for c in args.calls.split(",") if c)
+    if not set(args.calls) <= set(Step.ALL):
+        ap.error(f"--calls must be a subset of {Step.ALL}")
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
