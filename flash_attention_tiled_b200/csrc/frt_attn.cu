@@ -236,6 +236,35 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
+// ------------------------------------------- decode without caller scratch
+// Scratch of frt_attn_decode_paged_noalloc: one fixed buffer per device,
+// reserved when the library is loaded and held until the process exits.  In
+// host code this name only stands for the device variable; the kernel gets
+// its device address from cudaGetSymbolAddress, taken once per device.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;
+static __device__ __align__(256) unsigned char frt_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of this device's scratch (looked up on the first call made
+// with that device current).
+frt_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FRT_ERR_CUDA;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, frt_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return FRT_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+  }
+  *out = g_noalloc_ptr[dev];
+  return FRT_OK;
+}
+
 }  // namespace
 }  // namespace frt
 
@@ -324,6 +353,38 @@ frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_parts, int 
     merge_lse_kernel<64><<<(unsigned)blocks, kMergeWarps * 32, 0, stream>>>(
         o_parts, lse_parts, S, rows, static_cast<__nv_bfloat16*>(o), lse);
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pages,
+                                         const void* v_pages, const int32_t* block_table,
+                                         int max_pages_per_seq, const int32_t* seq_lens,
+                                         int page_size, int num_pages, void* o, float* lse,
+                                         int B, int Hq, int Hkv, int D, float scale,
+                                         int num_splits, cudaStream_t stream) {
+  // size this call needs, checked against the fixed scratch before anything runs
+  size_t need = 0;
+  frt_status st = frt_attn_decode_paged(nullptr, k_pages, v_pages, block_table,
+                                        max_pages_per_seq, seq_lens, page_size, num_pages, o,
+                                        lse, B, Hq, Hkv, D, scale, num_splits, nullptr, &need,
+                                        stream);
+  if (st != FRT_OK) return st;
+  if (need > kNoAllocScratchBytes) return FRT_ERR_WORKSPACE;
+  if (B == 0) return FRT_OK;
+  if (q == nullptr) return FRT_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != FRT_OK) return st;
+  // The scratch keeps whatever the previous call left there; the arrival
+  // counters at its start must read zero when the kernel begins.
+  const int g = Hkv > 0 ? Hq / Hkv : 0;
+  const size_t counter_bytes =
+      (size_t)B * Hkv * ((g + kDecHeadsPerSeg - 1) / kDecHeadsPerSeg) * sizeof(unsigned);
+  if (counter_bytes > 0 && cudaMemsetAsync(scratch, 0, counter_bytes, stream) != cudaSuccess)
+    return FRT_ERR_CUDA;
+  size_t have = kNoAllocScratchBytes;
+  return frt_attn_decode_paged(q, k_pages, v_pages, block_table, max_pages_per_seq, seq_lens,
+                               page_size, num_pages, o, lse, B, Hq, Hkv, D, scale, num_splits,
+                               scratch, &have, stream);
 }
 
 frt_status frt_read_device_error(unsigned* flags) {

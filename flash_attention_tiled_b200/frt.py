@@ -16,8 +16,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
-EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_merge_lse",
-           "frt_read_device_error", "frt_version")
+EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
+           "frt_attn_merge_lse", "frt_read_device_error", "frt_version")
 
 STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
           3: "FRT_ERR_WORKSPACE", 4: "FRT_ERR_CUDA"}
@@ -38,6 +38,8 @@ def _load() -> ctypes.CDLL:
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_size_t)
     lib.frt_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
     lib.frt_attn_decode_paged.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I, P, Z, P]
+    lib.frt_attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F,
+                                                  I, P]
     lib.frt_attn_merge_lse.argtypes = [P, P, I, I, I, I, P, P, P]
     lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     for name in EXPORTS[:-1]:
@@ -155,6 +157,35 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
         _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale, num_splits,
         _ptr(ws), ctypes.byref(need), stream))
+    return out, lse
+
+
+def attn_decode_paged_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                              block_table: torch.Tensor, seq_lens: torch.Tensor,
+                              scale: float | None = None, num_splits: int = 0,
+                              out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                              return_lse: bool = True):
+    """attn_decode_paged without a workspace: the library's fixed per-device
+    scratch buffer is used instead (see frt_attn_decode_paged_noalloc in
+    include/frt_attn.h for its size limit and the rule that calls which may
+    overlap on the device race)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check("frt_attn_decode_paged_noalloc", _lib.frt_attn_decode_paged_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale, num_splits,
+        _stream(q.device)))
     return out, lse
 
 

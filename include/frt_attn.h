@@ -139,6 +139,45 @@ FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, con
                                  size_t* workspace_bytes, cudaStream_t stream);
 
 /*
+ * frt_attn_decode_paged_noalloc -- frt_attn_decode_paged for callers that
+ * cannot allocate device memory.  No page describes this entry point; it is
+ * a convenience of this library.
+ *
+ * Who needs it: code whose device memory is planned once and must not call
+ * cudaMalloc while it runs -- an engine plugin handed fixed buffers, a
+ * real-time decode loop that cannot afford an allocation's implicit device
+ * synchronisation and unbounded latency, an embedded runtime with no
+ * allocator at hand.  Such a caller cannot provide frt_attn_decode_paged's
+ * workspace.
+ *
+ * What it does: the same computation, arguments and results as
+ * frt_attn_decode_paged, with the workspace taken from a fixed 16 MiB
+ * buffer that the library reserves in every GPU's memory when it is loaded
+ * (held until the process exits).  It allocates nothing and frees nothing.
+ *   - Limit: a problem whose workspace (see frt_attn_decode_paged's size
+ *     query) exceeds 16 MiB is rejected with FRT_ERR_WORKSPACE before
+ *     anything runs.  At D = 128 with one partition per SM that is roughly
+ *     B * Hkv <= 1800 (fewer when a KV head serves more than 16 query heads).
+ *   - The first call made with a given device current looks up that
+ *     device's buffer address; make that first call before any stream
+ *     capture on that device.
+ *   - Each call first clears the buffer's arrival counters on `stream`
+ *     (a memset of B * Hkv * ceil(Hq/Hkv/16) * 4 bytes), then launches.
+ *   - All calls on a device share the one buffer, and it keeps what the
+ *     last call left in it: calls that can overlap on the device (different
+ *     streams without ordering) race and corrupt each other's results.
+ *     Order them, or use frt_attn_decode_paged with separate workspaces.
+ */
+FRT_API frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pages,
+                                                 const void* v_pages,
+                                                 const int32_t* block_table,
+                                                 int max_pages_per_seq, const int32_t* seq_lens,
+                                                 int page_size, int num_pages, void* o,
+                                                 float* lse, int B, int Hq, int Hkv, int D,
+                                                 float scale, int num_splits,
+                                                 cudaStream_t stream);
+
+/*
  * frt_attn_merge_lse -- combine S partial attention results of the same rows,
  * each computed over a disjoint set of keys, into the result over their
  * union.  This is the correct form of the per-page combination in the
