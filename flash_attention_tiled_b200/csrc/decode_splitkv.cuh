@@ -22,11 +22,13 @@
 //
 // Inside a CTA: warp 0 streams pages into a ring of shared-memory stages with
 // TMA (128-byte swizzled 16x64 boxes, one mbarrier per stage), looking pages
-// up in the block table; warps 1..W each take one page of every stage and
-// compute S = Q.K^T and O += P.V with warp-level bf16 MMAs in which the
-// segment's query heads form the M dimension, so each K/V page is read from
-// HBM once for all heads of its group.  Scores live in the exp2 domain
-// (scale * log2(e) folded in); the online max/sum use quad shuffles.
+// up in the block table; warps 1..W each take two pages (32 tokens) of every
+// stage and compute S = Q.K^T and O += P.V with warp-level bf16 MMAs in which
+// the segment's query heads form the M dimension, so each K/V page is read
+// from HBM once for all heads of its group.  Scores live in the exp2 domain
+// (scale * log2(e) folded in); the online max/sum use quad shuffles.  At the
+// end of a piece the warps' states are combined in registers (two levels
+// through shared memory) and written by one warp.
 #pragma once
 
 #include "frt_device.cuh"
@@ -35,6 +37,8 @@ namespace frt {
 
 constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
 constexpr int kDecWarps = 4;          // consumer warps per CTA
+constexpr int kDecPagesPerWarp = 2;   // pages a consumer warp takes per stage
+constexpr int kDecStagePages = kDecWarps * kDecPagesPerWarp;
 constexpr int kDecThreads = 32 * (kDecWarps + 1);
 constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
 constexpr int kDecMaxBatch = 1024;    // prefix table held in shared memory
@@ -59,17 +63,19 @@ struct DecodeSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 64 bf16
   static constexpr int kPageBytes = kHalves * kBoxBytes;              // K or V of one page
-  static constexpr int kStageBytes = kDecWarps * 2 * kPageBytes;      // K+V of W pages
-  static constexpr int kStages = (D == 128) ? 5 : 10;
+  static constexpr int kStageBytes = kDecStagePages * 2 * kPageBytes; // K+V of 8 pages
+  static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kRingBytes = kStages * kStageBytes;
-  // cross-warp merge scratch: per warp m[16], l[16], l_exact[16], O[16][D]
-  static constexpr int kScratchStride = 3 * kDecHeadsPerSeg + kDecHeadsPerSeg * D;
-  static constexpr int kScratchFloats = kDecWarps * kScratchStride;
+  // cross-warp combine: one warp's register state in fragment order
+  // (D/8 output tiles x 4 accumulators, then m, l, l_exact for 2 row halves)
+  static constexpr int kFragFloats = (D / 8) * 4 + 6;
+  static constexpr int kScratchFloats = 2 * kFragFloats * 32;
   static constexpr int kScratchOff = kRingBytes;
   static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
   static constexpr int kBarOff = kPrefixOff + ((kDecMaxBatch + 1) * 4 + 15) / 16 * 16;
   static constexpr int kBytes = 1024 /*alignment slack*/ + kBarOff + 2 * kStages * 8;
   static_assert(kBarOff % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
 // Pages of sequence b (seq_len clamped to [0, max_pages * 16]).
@@ -230,8 +236,8 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     bool ok = true;
     do {
       const int kvh = pc.seg_in_b / p.hgroups;
-      for (int pb = pc.pg0; pb < pc.pg1 && ok; pb += kDecWarps) {
-        const int n = min(kDecWarps, pc.pg1 - pb);
+      for (int pb = pc.pg0; pb < pc.pg1 && ok; pb += kDecStagePages) {
+        const int n = min(kDecStagePages, pc.pg1 - pb);
         // row of the page's first token in the [rows, D] view of the cache
         int row = 0;
         if (lane < n) {
@@ -270,11 +276,9 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int cw = warp - 1;               // consumer warp index
   const int quad = lane >> 2;            // MMA row group: head rows quad, quad+8
   const int qc = lane & 3;               // column pair within the quad
-  float* my_m = scratch + cw * L::kScratchStride;
-  float* my_l = my_m + kDecHeadsPerSeg;
-  float* my_le = my_l + kDecHeadsPerSeg;
-  float* my_o = my_le + kDecHeadsPerSeg;
+  const int t0 = 2 * qc;                 // first token column of this lane in an 8-wide tile
   const uint32_t ring_u32 = smem_u32(ring);
+  constexpr float kLn2 = 0.69314718055994530942f;
 
   int stage = 0;
   uint32_t phase = 0;
@@ -308,91 +312,126 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
     for (int t = 0; t < kNTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
-    for (int pb = pc.pg0; pb < pc.pg1; pb += kDecWarps) {
+    for (int pb = pc.pg0; pb < pc.pg1; pb += kDecStagePages) {
       ok = mbar_wait_warp(&full_bar[stage], phase, &abort_flag);
       if (!ok) break;
-      const int page = pb + cw;
-      if (page < pc.pg1) {
-        const uint32_t kbase = ring_u32 + stage * L::kStageBytes + cw * 2 * L::kPageBytes;
-        const uint32_t vbase = kbase + L::kPageBytes;
-        const int valid = min(kDecPage, len - page * kDecPage);   // tokens of this page
+      const int page_a = pb + kDecPagesPerWarp * cw;     // this warp's two pages
+      const int valid_a = page_a < pc.pg1 ? min(kDecPage, len - page_a * kDecPage) : 0;
+      const int valid_b =
+          page_a + 1 < pc.pg1 ? min(kDecPage, len - (page_a + 1) * kDecPage) : 0;
+      if (valid_a > 0) {
+        const bool has_b = valid_b > 0;
+        const uint32_t ka = ring_u32 + stage * L::kStageBytes +
+                            kDecPagesPerWarp * cw * 2 * L::kPageBytes;
+        const uint32_t va = ka + L::kPageBytes;
+        const uint32_t kb = ka + 2 * L::kPageBytes;
+        const uint32_t vb = kb + L::kPageBytes;
 
-        // ---- S = Q.K^T: two 16x8 tiles (tokens 0-7, 8-15)
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S = Q.K^T: four 16x8 tiles (tokens 0-7, 8-15 of each page)
+        float s[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
         {
           const int mi = lane >> 3, r = lane & 7;
           const int tok = (mi >> 1) * 8 + r;
 #pragma unroll
           for (int ks = 0; ks < kKSteps; ++ks) {
             const int col = ks * 16 + (mi & 1) * 8;
-            const uint32_t addr =
-                sw128_addr(kbase + (col >> 6) * L::kBoxBytes, tok, col & 63);
+            const uint32_t off = (col >> 6) * L::kBoxBytes;
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(addr, b0, b1, b2, b3);
-            mma_bf16_16816(s0, qa[ks], b0, b1);
-            mma_bf16_16816(s1, qa[ks], b2, b3);
+            ldsm_x4(sw128_addr(ka + off, tok, col & 63), b0, b1, b2, b3);
+            mma_bf16_16816(s[0], qa[ks], b0, b1);
+            mma_bf16_16816(s[1], qa[ks], b2, b3);
+            if (has_b) {
+              ldsm_x4(sw128_addr(kb + off, tok, col & 63), b0, b1, b2, b3);
+              mma_bf16_16816(s[2], qa[ks], b0, b1);
+              mma_bf16_16816(s[3], qa[ks], b2, b3);
+            }
           }
         }
-        // ---- scores in the exp2 domain, tail tokens masked by select
-        const int t0 = 2 * qc;   // token of s0[0]; s0[1] -> t0+1; s1 -> +8
-        float sc[2][4];          // [row half][tok t0, t0+1, t0+8, t0+9]
+        // ---- scores in the exp2 domain; tokens past the sequence end -> -inf
+        // sc[rh][i]: row quad + 8*rh, token (page a) t0, t0+1, t0+8, t0+9,
+        // (page b) t0, t0+1, t0+8, t0+9
+        float sc[2][8];
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh) {
-          sc[rh][0] = (t0 < valid) ? s0[2 * rh] * p.scale_log2 : -INFINITY;
-          sc[rh][1] = (t0 + 1 < valid) ? s0[2 * rh + 1] * p.scale_log2 : -INFINITY;
-          sc[rh][2] = (t0 + 8 < valid) ? s1[2 * rh] * p.scale_log2 : -INFINITY;
-          sc[rh][3] = (t0 + 9 < valid) ? s1[2 * rh + 1] * p.scale_log2 : -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tok = t0 + (i & 1) + (i >> 1) * 8;
+            sc[rh][i] = (tok < valid_a) ? s[i >> 1][2 * rh + (i & 1)] * p.scale_log2 : -INFINITY;
+            sc[rh][4 + i] =
+                (tok < valid_b) ? s[2 + (i >> 1)][2 * rh + (i & 1)] * p.scale_log2 : -INFINITY;
+          }
         }
-        uint32_t pa[4];
+        uint32_t pa[4], pbv[4];   // P fragments of page a and page b
+        float alpha[2];
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh) {
-          float mx = fmaxf(fmaxf(sc[rh][0], sc[rh][1]), fmaxf(sc[rh][2], sc[rh][3]));
+          float mx = fmaxf(fmaxf(fmaxf(sc[rh][0], sc[rh][1]), fmaxf(sc[rh][2], sc[rh][3])),
+                           fmaxf(fmaxf(sc[rh][4], sc[rh][5]), fmaxf(sc[rh][6], sc[rh][7])));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
           const float m_new = fmaxf(m_run[rh], mx);
-          const float alpha = fast_exp2(m_run[rh] - m_new);   // 0 on the first page
+          alpha[rh] = fast_exp2(m_run[rh] - m_new);   // 0 on the first step
           m_run[rh] = m_new;
-          const float e0 = fast_exp2(sc[rh][0] - m_new), e1 = fast_exp2(sc[rh][1] - m_new);
-          const float e2 = fast_exp2(sc[rh][2] - m_new), e3 = fast_exp2(sc[rh][3] - m_new);
-          const uint32_t lo = pack_bf16x2(e0, e1);
-          const uint32_t hi = pack_bf16x2(e2, e3);
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) e[i] = fast_exp2(sc[rh][i] - m_new);
+          const uint32_t w0 = pack_bf16x2(e[0], e[1]), w1 = pack_bf16x2(e[2], e[3]);
+          const uint32_t w2 = pack_bf16x2(e[4], e[5]), w3 = pack_bf16x2(e[6], e[7]);
           // O is normalised by the bf16-rounded weights that feed P.V; the LSE
           // uses the exact ones
-          const float psum = __uint_as_float(lo << 16) + __uint_as_float(lo & 0xffff0000u) +
-                             __uint_as_float(hi << 16) + __uint_as_float(hi & 0xffff0000u);
-          l_run[rh] = l_run[rh] * alpha + psum;
-          le_run[rh] = le_run[rh] * alpha + ((e0 + e1) + (e2 + e3));
+          const float psum = (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u)) +
+                             (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u)) +
+                             (__uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xffff0000u)) +
+                             (__uint_as_float(w3 << 16) + __uint_as_float(w3 & 0xffff0000u));
+          const float esum = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+          l_run[rh] = l_run[rh] * alpha[rh] + psum;
+          le_run[rh] = le_run[rh] * alpha[rh] + esum;
+          pa[rh] = w0;        // a0a1 (rh=0) / a2a3 (rh=1): tokens t0, t0+1
+          pa[2 + rh] = w1;    // a4a5 / a6a7: tokens t0+8, t0+9
+          pbv[rh] = w2;
+          pbv[2 + rh] = w3;
+        }
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
           for (int t = 0; t < kNTiles; ++t) {
-            acc[t][2 * rh] *= alpha;
-            acc[t][2 * rh + 1] *= alpha;
+            acc[t][0] *= alpha[0];
+            acc[t][1] *= alpha[0];
+            acc[t][2] *= alpha[1];
+            acc[t][3] *= alpha[1];
           }
-          pa[rh] = lo;        // a0a1 (rh=0) / a2a3 (rh=1): tokens t0, t0+1
-          pa[2 + rh] = hi;    // a4a5 / a6a7: tokens t0+8, t0+9
         }
         // ---- O += P.V: V^T fragments by transposing ldmatrix
         {
           const int mi = lane >> 3, r = lane & 7;
           const int tok = (mi & 1) * 8 + r;
-          // B-fragment halves: b0b1 -> tokens 2qc, 2qc+1; b2b3 -> +8
-          const bool kill_lo0 = t0 >= valid, kill_hi0 = t0 + 1 >= valid;
-          const bool kill_lo1 = t0 + 8 >= valid, kill_hi1 = t0 + 9 >= valid;
-          const bool tail = valid < kDecPage;
+          const bool tail_a = valid_a < kDecPage, tail_b = has_b && valid_b < kDecPage;
 #pragma unroll
           for (int nt = 0; nt < kNTiles; nt += 2) {
             const int col = (nt + (mi >> 1)) * 8;
-            const uint32_t addr =
-                sw128_addr(vbase + (col >> 6) * L::kBoxBytes, tok, col & 63);
+            const uint32_t off = (col >> 6) * L::kBoxBytes;
             uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(addr, b0, b1, b2, b3);
-            if (tail) {   // tokens past the sequence end may hold anything (NaN)
-              b0 = (kill_lo0 ? 0u : (b0 & 0xffffu)) | (kill_hi0 ? 0u : (b0 & 0xffff0000u));
-              b2 = (kill_lo0 ? 0u : (b2 & 0xffffu)) | (kill_hi0 ? 0u : (b2 & 0xffff0000u));
-              b1 = (kill_lo1 ? 0u : (b1 & 0xffffu)) | (kill_hi1 ? 0u : (b1 & 0xffff0000u));
-              b3 = (kill_lo1 ? 0u : (b3 & 0xffffu)) | (kill_hi1 ? 0u : (b3 & 0xffff0000u));
+            ldsm_x4_trans(sw128_addr(va + off, tok, col & 63), b0, b1, b2, b3);
+            if (tail_a) {   // tokens past the sequence end may hold anything (NaN)
+              b0 = (t0 < valid_a ? (b0 & 0xffffu) : 0u) | (t0 + 1 < valid_a ? (b0 & 0xffff0000u) : 0u);
+              b2 = (t0 < valid_a ? (b2 & 0xffffu) : 0u) | (t0 + 1 < valid_a ? (b2 & 0xffff0000u) : 0u);
+              b1 = (t0 + 8 < valid_a ? (b1 & 0xffffu) : 0u) | (t0 + 9 < valid_a ? (b1 & 0xffff0000u) : 0u);
+              b3 = (t0 + 8 < valid_a ? (b3 & 0xffffu) : 0u) | (t0 + 9 < valid_a ? (b3 & 0xffff0000u) : 0u);
             }
             mma_bf16_16816(acc[nt], pa, b0, b1);
             mma_bf16_16816(acc[nt + 1], pa, b2, b3);
+            if (has_b) {
+              ldsm_x4_trans(sw128_addr(vb + off, tok, col & 63), b0, b1, b2, b3);
+              if (tail_b) {
+                b0 = (t0 < valid_b ? (b0 & 0xffffu) : 0u) | (t0 + 1 < valid_b ? (b0 & 0xffff0000u) : 0u);
+                b2 = (t0 < valid_b ? (b2 & 0xffffu) : 0u) | (t0 + 1 < valid_b ? (b2 & 0xffff0000u) : 0u);
+                b1 = (t0 + 8 < valid_b ? (b1 & 0xffffu) : 0u) | (t0 + 9 < valid_b ? (b1 & 0xffff0000u) : 0u);
+                b3 = (t0 + 8 < valid_b ? (b3 & 0xffffu) : 0u) | (t0 + 9 < valid_b ? (b3 & 0xffff0000u) : 0u);
+              }
+              mma_bf16_16816(acc[nt], pbv, b0, b1);
+              mma_bf16_16816(acc[nt + 1], pbv, b2, b3);
+            }
           }
         }
       }
@@ -401,100 +440,140 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
       if (++stage == kStages) { stage = 0; phase ^= 1u; }
     }
 
-    // ---- this warp's state -> scratch
-#pragma unroll
-    for (int rh = 0; rh < 2; ++rh) {
-      float ls = l_run[rh], le = le_run[rh];
-      ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-      ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-      le += __shfl_xor_sync(0xffffffffu, le, 1);
-      le += __shfl_xor_sync(0xffffffffu, le, 2);
-      if (qc == 0) {
-        my_m[quad + 8 * rh] = m_run[rh];
-        my_l[quad + 8 * rh] = ls;
-        my_le[quad + 8 * rh] = le;
-      }
-#pragma unroll
-      for (int t = 0; t < kNTiles; ++t) {
-        float2 v2 = make_float2(acc[t][2 * rh], acc[t][2 * rh + 1]);
-        *reinterpret_cast<float2*>(&my_o[(quad + 8 * rh) * D + t * 8 + 2 * qc]) = v2;
-      }
-    }
+    // ---- combine the four warps' states in registers: 2,3 -> 0,1 -> 0
     // stop together if any warp gave up (every consumer gets the same answer)
     if (bar_sync_or(1, kDecWarps * 32, !ok || abort_flag)) break;
+#pragma unroll
+    for (int level = 0; level < 2; ++level) {
+      const int senders = level == 0 ? 2 : 1;        // warps [senders, 2*senders) send
+      if (cw >= senders && cw < 2 * senders) {
+        float* dst = scratch + (cw - senders) * L::kFragFloats * 32 + lane;
+#pragma unroll
+        for (int t = 0; t < kNTiles; ++t)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[(t * 4 + i) * 32] = acc[t][i];
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          dst[(kNTiles * 4 + rh) * 32] = m_run[rh];
+          dst[(kNTiles * 4 + 2 + rh) * 32] = l_run[rh];
+          dst[(kNTiles * 4 + 4 + rh) * 32] = le_run[rh];
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
+      if (cw < senders) {
+        const float* src = scratch + cw * L::kFragFloats * 32 + lane;
+        float wa[2], wb[2];
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          const float mo = src[(kNTiles * 4 + rh) * 32];
+          const float mn = fmaxf(m_run[rh], mo);
+          // a state that saw no key has m = -inf and contributes nothing
+          wa[rh] = (m_run[rh] == -INFINITY) ? 0.f : fast_exp2(m_run[rh] - mn);
+          wb[rh] = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+          m_run[rh] = mn;
+          l_run[rh] = l_run[rh] * wa[rh] + src[(kNTiles * 4 + 2 + rh) * 32] * wb[rh];
+          le_run[rh] = le_run[rh] * wa[rh] + src[(kNTiles * 4 + 4 + rh) * 32] * wb[rh];
+        }
+#pragma unroll
+        for (int t = 0; t < kNTiles; ++t)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            acc[t][i] = acc[t][i] * wa[i >> 1] + src[(t * 4 + i) * 32] * wb[i >> 1];
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
+    }
 
-    // ---- combine the warps: one partial (or the final result) per piece
+    // ---- warp 0 writes the piece: the final rows, or one partial
     const int seg = pc.b * nseg_b + pc.seg_in_b;
     const bool whole = (pc.pg0 == 0) && (pc.pg1 == pc.npg);
     const int slot = c + seg;
-    const int ct = threadIdx.x - 32;
-    constexpr int kStride = L::kScratchStride;
-    for (int e = ct; e < nh * D; e += kDecWarps * 32) {
-      const int r = e / D, d = e % D;
-      float M = -INFINITY;
+    if (cw == 0) {
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, scratch[w * kStride + r]);
-      float Lsum = 0.f, Lexact = 0.f, Osum = 0.f;
+      for (int rh = 0; rh < 2; ++rh) {
+        float ls = l_run[rh], le = le_run[rh];
+        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+        le += __shfl_xor_sync(0xffffffffu, le, 1);
+        le += __shfl_xor_sync(0xffffffffu, le, 2);
+        const int r = quad + 8 * rh;
+        if (r < nh) {
+          const float inv = 1.f / ls;
+          const float lse2 = m_run[rh] + fast_log2(le);
+          if (whole) {
+            __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float* sw = scratch + w * kStride;
-        const float mw = sw[r];
-        const float wgt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        Lsum += wgt * sw[kDecHeadsPerSeg + r];
-        Lexact += wgt * sw[2 * kDecHeadsPerSeg + r];
-        Osum += wgt * sw[3 * kDecHeadsPerSeg + r * D + d];
+            for (int t = 0; t < kNTiles; ++t)
+              *reinterpret_cast<uint32_t*>(orow + t * 8 + t0) =
+                  pack_bf16x2(acc[t][2 * rh] * inv, acc[t][2 * rh + 1] * inv);
+            if (qc == 0 && p.lse != nullptr) p.lse[(size_t)pc.b * p.Hq + h0 + r] = lse2 * kLn2;
+          } else {
+            float* orow = p.ws_o + ((size_t)slot * kDecHeadsPerSeg + r) * D;
+#pragma unroll
+            for (int t = 0; t < kNTiles; ++t)
+              *reinterpret_cast<float2*>(orow + t * 8 + t0) =
+                  make_float2(acc[t][2 * rh] * inv, acc[t][2 * rh + 1] * inv);
+            if (qc == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
+          }
+        }
       }
-      const float o_val = Osum / Lsum;
-      const float lse2 = M + fast_log2(Lexact);
-      if (whole) {
-        const size_t row = (size_t)pc.b * p.Hq + h0 + r;
-        p.o[row * D + d] = __float2bfloat16(o_val);
-        if (d == 0 && p.lse != nullptr) p.lse[row] = lse2 * 0.69314718055994530942f;
-      } else {
-        p.ws_o[((size_t)slot * kDecHeadsPerSeg + r) * D + d] = o_val;
-        if (d == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
+      if (!whole) {
+        // ticket: the last piece of this segment to finish merges all of them
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          const int c_first = dec_cta_of(pc.seg_u0, T, C);
+          const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C);
+          const unsigned parts = (unsigned)(c_last - c_first + 1);
+          const unsigned prev = atomicAdd(&p.ws_count[seg], 1u);
+          if (prev == parts - 1) {
+            p.ws_count[seg] = 0u;   // ready for the next call
+            __threadfence();
+            last = c_first + 1;
+          }
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (lane == 0) s_is_last = last;
       }
     }
     if (!whole) {
-      // ticket: the last piece of this segment to finish merges all of them
-      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
-      if (ct == 0) {
-        __threadfence();
-        const long long T_ = T;
-        const int c_first = dec_cta_of(pc.seg_u0, T_, C);
-        const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T_, C);
-        const unsigned parts = (unsigned)(c_last - c_first + 1);
-        const unsigned prev = atomicAdd(&p.ws_count[seg], 1u);
-        s_is_last = (prev == parts - 1) ? (c_first + 1) : 0;   // store c_first + 1
-        if (prev == parts - 1) {
-          p.ws_count[seg] = 0u;   // ready for the next call
-          __threadfence();
-        }
-      }
       asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
       if (s_is_last) {
+        // single pass over the parts with a running maximum; every thread
+        // owns 4 consecutive d of one row, loads of later parts overlap
         const int c_first = s_is_last - 1;
         const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C);
-        for (int e = ct; e < nh * D; e += kDecWarps * 32) {
-          const int r = e / D, d = e % D;
-          float M = -INFINITY;
-          for (int cc = c_first; cc <= c_last; ++cc)
-            M = fmaxf(M, __ldcg(&p.ws_lse[(size_t)(cc + seg) * kDecHeadsPerSeg + r]));
-          float Lsum = 0.f, Osum = 0.f;
+        const int ct = threadIdx.x - 32;
+        for (int e = ct; e < nh * (D / 4); e += kDecWarps * 32) {
+          const int r = e / (D / 4), d4 = (e % (D / 4)) * 4;
+          float M = -INFINITY, S = 0.f;
+          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
           for (int cc = c_first; cc <= c_last; ++cc) {
             const size_t sl = (size_t)(cc + seg);
-            const float wgt = fast_exp2(__ldcg(&p.ws_lse[sl * kDecHeadsPerSeg + r]) - M);
-            Lsum += wgt;
-            Osum += wgt * __ldcg(&p.ws_o[(sl * kDecHeadsPerSeg + r) * D + d]);
+            const float x = __ldcg(&p.ws_lse[sl * kDecHeadsPerSeg + r]);
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                &p.ws_o[(sl * kDecHeadsPerSeg + r) * D + d4]));
+            const float mn = fmaxf(M, x);
+            const float a = fast_exp2(M - mn);   // 0 while M = -inf
+            const float w = fast_exp2(x - mn);
+            S = S * a + w;
+            o4.x = o4.x * a + w * v.x;
+            o4.y = o4.y * a + w * v.y;
+            o4.z = o4.z * a + w * v.z;
+            o4.w = o4.w * a + w * v.w;
+            M = mn;
           }
-          const size_t row = (size_t)pc.b * p.Hq + h0 + r;
-          p.o[row * D + d] = __float2bfloat16(Osum / Lsum);
-          if (d == 0 && p.lse != nullptr)
-            p.lse[row] = (M + fast_log2(Lsum)) * 0.69314718055994530942f;
+          const float inv = 1.f / S;
+          __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D + d4;
+          *reinterpret_cast<uint2*>(orow) =
+              make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
+          if (d4 == 0 && p.lse != nullptr)
+            p.lse[(size_t)pc.b * p.Hq + h0 + r] = (M + fast_log2(S)) * kLn2;
         }
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch reuse
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch, s_is_last reuse
   } while (next_piece(pc));
 }
 

@@ -251,19 +251,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       const int kv0 = j * kPfBN;
       const bool need_mask = (p.causal && kv0 + kPfBN - 1 > q0 + off) || (kv0 + kPfBN > p.Skv);
-      float mx = -INFINITY;
       if (need_mask) {
         long long cmax = row_lim - kv0;
         const long long tail = (long long)p.Skv - 1 - kv0;
         if (tail < cmax) cmax = tail;
 #pragma unroll
-        for (int c = 0; c < kPfBN; ++c) {
-          s[c] = (c <= cmax) ? s[c] : -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
+        for (int c = 0; c < kPfBN; ++c) s[c] = (c <= cmax) ? s[c] : -INFINITY;
+      }
+      // row max: four independent three-input chains
+      float mx;
+      {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kPfBN; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kPfBN; c += 8) {
+          m0 = max3f(m0, s[c], s[c + 1]);
+          m1 = max3f(m1, s[c + 2], s[c + 3]);
+          m2 = max3f(m2, s[c + 4], s[c + 5]);
+          m3 = max3f(m3, s[c + 6], s[c + 7]);
+        }
+        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
       }
       const float m_tile = mx * p.scale_log2;
       // move the reference only when the max grew by more than the threshold
@@ -293,20 +299,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // P = exp2(s * scale_log2 - m_ref), rounded to bf16, written over S
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
       uint32_t pk[kPfBN / 2];
-      float rsum = 0.f, esum = 0.f;
+      {
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t ref2 = f2_pack(neg_ref, neg_ref);
+        uint64_t rs0 = 0, rs1 = 0, es0 = 0, es1 = 0;   // packed partial sums (0.0f pairs)
 #pragma unroll
-      for (int c = 0; c < kPfBN; c += 2) {
-        const float e0 = fast_exp2(fmaf(s[c], p.scale_log2, neg_ref));
-        const float e1 = fast_exp2(fmaf(s[c + 1], p.scale_log2, neg_ref));
-        const uint32_t w = pack_bf16x2(e0, e1);
-        pk[c / 2] = w;
-        // O is normalised by the same rounded weights that feed P.V, so that
-        // it stays a convex combination of V rows; the LSE uses the exact sum
-        rsum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
-        esum += e0 + e1;
+        for (int c = 0; c < kPfBN; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, ref2), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          const uint32_t w = pack_bf16x2(e0, e1);
+          pk[c / 2] = w;
+          // O is normalised by the same rounded weights that feed P.V, so that
+          // it stays a convex combination of V rows; the LSE uses the exact sum
+          const uint64_t wr = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+          const uint64_t we = f2_pack(e0, e1);
+          if ((c & 2) == 0) { rs0 = f2_add(rs0, wr); es0 = f2_add(es0, we); }
+          else              { rs1 = f2_add(rs1, wr); es1 = f2_add(es1, we); }
+        }
+        float a, b2, c2, d2;
+        f2_unpack(f2_add(rs0, rs1), a, b2);
+        f2_unpack(f2_add(es0, es1), c2, d2);
+        l_sum += a + b2;
+        l_exact += c2 + d2;
       }
-      l_sum += rsum;
-      l_exact += esum;
       tmem_st32(s_addr, pk);
       tmem_st32(s_addr + 32, pk + 32);
       tc_wait_st();
