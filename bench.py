@@ -223,14 +223,23 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.graph(g_step, stream=stream):
         for n in names:
             st.call(n)
+    # Per-call timing graphs: R x (L2 flush, call) and R x (L2 flush) alone;
+    # a call's device time is the difference divided by R, so neither the
+    # graph launch nor the flush is counted.
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+    R = 20
+    g_flush = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_flush, stream=stream):
+        for _ in range(R):
+            flush.fill_(1.0)
     g_call = {}
     for n in names:
         g_call[n] = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_call[n], stream=stream):
-            st.call(n)
-    # L2 flush for the per-call timings: write twice the L2 size
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+            for _ in range(R):
+                flush.fill_(1.0)
+                st.call(n)
     with torch.cuda.stream(stream):
         for _ in range(3):
             g_step.replay()
@@ -258,26 +267,28 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
 
     # per-call device time, each call starting with a flushed L2
-    reps = max(3, min(args.steps, 50))
-    per_call_ms = {}
-    with torch.cuda.stream(stream):
-        for n in names:
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(reps)]
-            for a, b in evs:
-                flush.fill_(1.0)
+    def graph_ms(g, reps=5):
+        ts = []
+        with torch.cuda.stream(stream):
+            g.replay()
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                g_call[n].replay()
+                g.replay()
                 b.record(stream)
+                ts.append((a, b))
             torch.cuda.synchronize(device)
-            per_call_ms[n] = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        return float(np.median([a.elapsed_time(b) for a, b in ts]))
+
+    t_flush = graph_ms(g_flush)
+    per_call_ms = {n: max(graph_ms(g_call[n]) - t_flush, 1e-6) / R for n in names}
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         with torch.cuda.stream(stream):
             e2e = run_e2e(st, args, device)
-    del g_step, g_call
+    del g_step, g_call, g_flush
 
     if rank != 0:
         return None
@@ -340,7 +351,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
                    "parallelism": f"replicas x{world}",
                    "timing": "step = one CUDA graph of the four calls, replayed K times; "
-                             "per-call times: each call's own graph after an L2 flush",
+                             "per-call times: a graph of 20 x (L2 flush, call) minus a "
+                             "graph of 20 flushes, divided by 20",
                    "l2": "step working set ~0.9 GB > 126 MB L2 and every call's inputs are "
                          "evicted by the calls before it; per-call timings flush L2 "
                          "(2x L2 size written) before each call"},

@@ -21,7 +21,8 @@
 // segment; no CTA ever waits for another).
 //
 // Inside a CTA: warp 0 streams pages into a ring of shared-memory stages with
-// TMA (128-byte swizzled 16x64 boxes, one mbarrier per stage), looking pages
+// TMA (one 128-byte swizzled box per page and matrix, one mbarrier per
+// stage), looking pages
 // up in the block table; warps 1..W each take two pages (32 tokens) of every
 // stage and compute S = Q.K^T and O += P.V with warp-level bf16 MMAs in which
 // the segment's query heads form the M dimension, so each K/V page is read
@@ -113,7 +114,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using L = DecodeSmem<D>;
-  constexpr int kHalves = L::kHalves;
   constexpr int kStages = L::kStages;
   constexpr int kKSteps = D / 16;     // MMA K-steps of Q.K^T
   constexpr int kNTiles = D / 8;      // 8-wide output tiles of P.V
@@ -256,11 +256,8 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (lane < n) {
           uint8_t* kdst = ring + stage * L::kStageBytes + lane * 2 * L::kPageBytes;
           uint8_t* vdst = kdst + L::kPageBytes;
-#pragma unroll
-          for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(kdst + h * L::kBoxBytes, &tmap_k, &full_bar[stage], h * 64, row);
-            tma_load_2d(vdst + h * L::kBoxBytes, &tmap_v, &full_bar[stage], h * 64, row);
-          }
+          tma_load_3d(kdst, &tmap_k, &full_bar[stage], 0, row, 0);
+          tma_load_3d(vdst, &tmap_v, &full_bar[stage], 0, row, 0);
         }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }

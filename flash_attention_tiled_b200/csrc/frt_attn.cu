@@ -27,6 +27,7 @@ constexpr int kMaxDevices = 64;
 // ------------------------------------------------------- device properties
 struct DeviceInfo {
   int sm_count = 0;
+  bool prefill_ok = false;   // register pool of the prefill launch covers its split
   bool kernels_configured = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -54,6 +55,15 @@ frt_status device_info(DeviceInfo** out) {
           cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrefillSmem<64>::kBytes) != cudaSuccess)
         return FRT_ERR_CUDA;
+      // The prefill kernel hands registers from its producer warpgroup to
+      // its softmax warpgroups (setmaxnreg).  That only works if the launch
+      // reserves exactly the pool the split adds up to; otherwise the
+      // increase would wait forever, so the kernel is never launched.
+      cudaFuncAttributes fa128, fa64;
+      if (cudaFuncGetAttributes(&fa128, prefill_kernel<128>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa64, prefill_kernel<64>) != cudaSuccess)
+        return FRT_ERR_CUDA;
+      di.prefill_ok = fa128.numRegs == kPfRegsLaunch && fa64.numRegs == kPfRegsLaunch;
       di.kernels_configured = true;
     }
   }
@@ -158,12 +168,15 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       !aligned16(workspace))
     return FRT_ERR_WORKSPACE;
 
+  // One TMA box per page: (64 columns, 16 rows, D/64 column halves).  The
+  // half index is the outermost box dimension, so the page lands in shared
+  // memory as D/64 consecutive 16x64 swizzled blocks.
   CUtensorMap tk, tv;
-  const uint64_t dims[2] = {(uint64_t)D, cache_rows};
-  const uint64_t strides[1] = {(uint64_t)D * 2};
-  const uint32_t box[2] = {64, (uint32_t)kDecPage};
-  if (!make_tmap(&tk, k_base, 2, dims, strides, box) ||
-      !make_tmap(&tv, v_base, 2, dims, strides, box))
+  const uint64_t dims[3] = {64, cache_rows, (uint64_t)(D / 64)};
+  const uint64_t strides[2] = {(uint64_t)D * 2, 128};
+  const uint32_t box[3] = {64, (uint32_t)kDecPage, (uint32_t)(D / 64)};
+  if (!make_tmap(&tk, k_base, 3, dims, strides, box) ||
+      !make_tmap(&tv, v_base, 3, dims, strides, box))
     return FRT_ERR_CUDA;
 
   DecodeParams p;
@@ -199,8 +212,9 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   DeviceInfo* di = nullptr;
   frt_status st = device_info(&di);
   if (st != FRT_OK) return st;
-  const int n_qtiles = (Sq + kPfBM - 1) / kPfBM;
-  if (n_qtiles > 65535) return FRT_ERR_UNSUPPORTED;
+  if (!di->prefill_ok) return FRT_ERR_UNSUPPORTED;
+  const int n_blocks = (Sq + kPfRows - 1) / kPfRows;
+  if (n_blocks > 65535) return FRT_ERR_UNSUPPORTED;
   // With Skv == 0 every tile has no key tile to visit (o = 0, lse = -inf);
   // the K/V maps then only need to be valid descriptors, never read.
   const void* kb = Skv > 0 ? k : q;
@@ -218,7 +232,6 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
     return FRT_ERR_CUDA;
   PrefillParams p;
   p.lse = lse;
-  p.o = static_cast<__nv_bfloat16*>(o);
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -226,9 +239,9 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.Sq = Sq;
   p.Skv = Skv;
   p.causal = causal;
-  p.n_qtiles = n_qtiles;
+  p.n_blocks = n_blocks;
   p.scale_log2 = scale * kLog2e;
-  const dim3 grid((unsigned)(B * Hq), (unsigned)n_qtiles);
+  const dim3 grid((unsigned)(B * Hq), (unsigned)n_blocks);
   if (D == 128)
     prefill_kernel<128><<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
   else

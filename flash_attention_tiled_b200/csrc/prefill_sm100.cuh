@@ -3,29 +3,33 @@
 //
 // What it computes is the FlashAttention-style forward of the "Real-time
 // inference optimisation" page (llmapi-app.pages.dev), section "Flash
-// Attention optimisation": for each 128-query tile, loop over 128-key tiles,
+// Attention optimisation": for each query tile, loop over 128-key tiles,
 // S = Q.K^T, online softmax (running max and sum, accumulator rescaled when
 // the max moves), O += P.V, finally O / l; plus causal masking and MQA/GQA
 // from the "FlashRT-HF-kernels" page (zingnex.cn), section "Attention
 // optimisation".  Key tiles that the causal mask hides completely are never
 // loaded or multiplied.
 //
-// Roles (one CTA = one 128-query tile of one query head, 6 warps):
-//   warp 0    TMA producer: Q once, then K and V tiles into a ring of
-//             shared-memory slots in the order the MMA warp consumes them
-//             (K0, K1, V0, K2, V1, ...), 128-byte swizzled.
-//   warp 1    allocates tensor memory and issues the MMAs from one thread:
-//             S_j = Q.K_j^T into one of two S buffers (TMEM, fp32), then
-//             O += P_j.V_j with P_j read from TMEM (it overwrites S_j as
-//             bf16) and O accumulating in TMEM.
-//   warps 2-5 softmax: each thread owns one query row (= one TMEM lane);
-//             it reads its S row, masks, keeps the running max and sum in
-//             the exp2 domain (scale*log2(e) folded in), writes P back to
-//             TMEM and rescales O in TMEM when needed; then the epilogue
-//             (O / l -> bf16 -> shared memory -> TMA store, and the LSE).
-// Rescaling is lazy: the exponent reference only moves when the row max
-// grows by more than 2^8, so O is rarely touched; the result is exact either
-// way because numerator and denominator share the reference.
+// One CTA owns two 128-row query tiles (A = rows 0-127, B = rows 128-255 of a
+// 256-row block of one head) that share every K/V tile.  Tensor memory holds
+// S_A, S_B (128 fp32 columns each) and O_A, O_B (D columns each); P_X is
+// written back over S_X as bf16 and is the A operand of O_X += P_X.V.
+// Roles (12 warps):
+//   warp 0      TMA producer: Q_A and Q_B once, then K_j, V_j into a ring of
+//               shared-memory slots (128-byte swizzled).
+//   warp 1      allocates tensor memory and issues every MMA from one
+//               thread, in the order PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1):
+//               while one tile's softmax runs, the other tile's MMAs keep the
+//               tensor cores busy.
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query row
+//               per thread (= one TMEM lane); exp2 domain (scale*log2(e)
+//               folded in); then the epilogue (O / l -> bf16 -> shared memory
+//               -> TMA store, and the LSE).
+// The producer/MMA warpgroup gives registers to the two softmax warpgroups
+// (setmaxnreg): 128 x 88 + 256 x 208 = 384 x 168 registers, the launch's pool.
+// Rescaling is lazy: the exponent reference only moves when the row max grows
+// by more than 2^8, so O is rarely touched; the result is exact either way
+// because numerator and denominator share the reference.
 #pragma once
 
 #include "frt_device.cuh"
@@ -34,31 +38,39 @@ namespace frt {
 
 constexpr int kPfBM = 128;             // query rows per tile (TMEM lanes)
 constexpr int kPfBN = 128;             // keys per tile
-constexpr int kPfThreads = 192;
+constexpr int kPfTiles = 2;            // query tiles per CTA
+constexpr int kPfRows = kPfBM * kPfTiles;
+constexpr int kPfThreads = 384;
+constexpr int kPfRegsLaunch = 168;     // 65536 / 384, rounded down to a multiple of 8
+constexpr int kPfRegsProducer = 88;    // warpgroup 0 after setmaxnreg.dec
+constexpr int kPfRegsSoftmax = 208;    // warpgroups 1, 2 after setmaxnreg.inc
+static_assert(128 * kPfRegsProducer + 256 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
+              "register split must fit in the launch's register pool");
 constexpr float kPfRescaleThreshold = 8.0f;   // log2 units
 
 template <int D>
 struct PrefillSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = 128 * 128;              // 128 rows x 64 bf16
-  static constexpr int kTileBytes = kHalves * kHalfBytes;   // Q, K or V tile
-  // K/V ring; D=64 keeps 8 slots so that one CTA fills the SM (the kernel
-  // allocates all 512 TMEM columns, so a second resident CTA would only wait)
-  static constexpr int kSlots = (D == 128) ? 4 : 8;
-  static constexpr int kQOff = 0;
-  static constexpr int kRingOff = kTileBytes;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;   // a Q, K or V tile
+  static constexpr int kSlots = (D == 128) ? 4 : 6;         // K/V ring
+  static constexpr int kQOff = 0;                           // Q_A, Q_B
+  static constexpr int kRingOff = kPfTiles * kTileBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 3 * kPfTiles + 1;
   static constexpr int kBytes = 1024 + kBarOff + kNumBars * 8 + 64;
-  // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D)
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+  // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B after it
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  __device__ static constexpr uint32_t col_s(int t) { return t ? kColS1 : kColS0; }
+  __device__ static constexpr uint32_t col_o(int t) { return t ? kColO1 : kColO0; }
 };
 
 struct PrefillParams {
   float* lse;          // [B, Hq, Sq] or nullptr
-  __nv_bfloat16* o;    // [B, Hq, Sq, D] (used only to zero rows without keys)
-  int B, Hq, Hkv, g, Sq, Skv, causal, n_qtiles;
+  int B, Hq, Hkv, g, Sq, Skv, causal, n_blocks;   // n_blocks = ceil(Sq / 256)
   float scale_log2;
 };
 
@@ -80,31 +92,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* q_full = bars;
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = ring_full + kSlots;
-  uint64_t* s_full = ring_empty + kSlots;     // [2]
-  uint64_t* p_full = s_full + 2;              // [2]
-  // pv_done[b]: PV_j with j % 2 == b completed.  One barrier per S buffer, so
-  // that a waiter never falls two phases behind (a parity wait on a barrier
-  // that completed twice since would return at once).
-  uint64_t* pv_done = p_full + 2;             // [2]
-  uint64_t* mma_drain = pv_done + 2;
+  uint64_t* s_full = ring_empty + kSlots;     // [tile]: QK_X(j) completed
+  uint64_t* p_full = s_full + kPfTiles;       // [tile]: P_X(j) written (128 arrivals)
+  uint64_t* pv_done = p_full + kPfTiles;      // [tile]: PV_X(j) completed
+  uint64_t* mma_drain = pv_done + kPfTiles;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- tile coordinates (heaviest causal tiles are scheduled first)
+  // ---- block coordinates (heaviest causal blocks are scheduled first)
   const int bh = blockIdx.x;                 // b * Hq + hq
-  const int qt = p.causal ? (p.n_qtiles - 1 - (int)blockIdx.y) : (int)blockIdx.y;
+  const int blk = p.causal ? (p.n_blocks - 1 - (int)blockIdx.y) : (int)blockIdx.y;
   const int b = bh / p.Hq, hq = bh % p.Hq;
   const int kv_row = b * p.Hkv + hq / p.g;   // z coordinate in the K/V maps
-  const int q0 = qt * kPfBM;
+  const int q_blk = blk * kPfRows;           // first query row of tile A
   const int off = p.Skv - p.Sq;              // bottom-right causal alignment
-  const int q_last = min(q0 + kPfBM - 1, p.Sq - 1);
+  const int q_last = min(q_blk + kPfRows - 1, p.Sq - 1);
   const int n_kv_all = (p.Skv + kPfBN - 1) / kPfBN;
   int n_kv = n_kv_all;
   if (p.causal) {
-    const int lim = q_last + off;            // largest key any row of the tile sees
+    const int lim = q_last + off;            // largest key any row of the block sees
     n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kPfBN + 1);
   }
 
@@ -114,10 +123,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&pv_done[s], 1);
+    for (int t = 0; t < kPfTiles; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(mma_drain, 1);
     abort_flag = 0;
@@ -132,39 +141,39 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 0) {
-    // ================================================= TMA producer
-    if (lane == 0 && n_kv > 0) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfRegsProducer));
+    if (warp == 0 && lane == 0 && n_kv > 0) {
+      // ================================================= TMA producer
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, L::kTileBytes);
+      mbar_arrive_expect_tx(q_full, kPfTiles * L::kTileBytes);
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h)
-        tma_load_3d(sq + h * L::kHalfBytes, &tm_q, q_full, h * 64, q0, bh);
+      for (int t = 0; t < kPfTiles; ++t)
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h)
+          tma_load_3d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
+                      q_blk + t * kPfBM, bh);
       int slot = 0;
       uint32_t phase = 0;
-      auto load = [&](const CUtensorMap* tm, int j) -> bool {
-        if (!mbar_wait(&ring_empty[slot], phase ^ 1u, &abort_flag)) return false;
+      bool ok = true;
+      // consumption order of the MMA warp: K0, V0, K1, V1, ...
+      for (int it = 0; it < 2 * n_kv && ok; ++it) {
+        const int j = it >> 1;
+        const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
+        ok = mbar_wait(&ring_empty[slot], phase ^ 1u, &abort_flag);
+        if (!ok) break;
         mbar_arrive_expect_tx(&ring_full[slot], L::kTileBytes);
         uint8_t* dst = ring + slot * L::kTileBytes;
 #pragma unroll
         for (int h = 0; h < kHalves; ++h)
           tma_load_3d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN, kv_row);
         if (++slot == kSlots) { slot = 0; phase ^= 1u; }
-        return true;
-      };
-      // the MMA warp consumes K0, then for each j: K_{j+1} (if any), V_j
-      bool ok = load(&tm_k, 0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv) ok = load(&tm_k, j + 1);
-        if (ok) ok = load(&tm_v, j);
       }
       if (!ok) __nanosleep(100000);
-    }
-  } else if (warp == 1) {
-    // ===================================================== MMA issuer
-    if (lane == 0 && n_kv > 0) {
+    } else if (warp == 1 && lane == 0 && n_kv > 0) {
+      // ===================================================== MMA issuer
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kPfBM, kPfBN, false, false);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(kPfBM, D, false, true);
       const uint32_t sq_addr = smem_u32(sq);
@@ -173,75 +182,106 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       uint32_t phase = 0;
       bool ok = mbar_wait(q_full, 0, &abort_flag);
 
-      auto issue_qk = [&](int sbuf) {
-        const uint32_t k_addr = ring_addr + slot * L::kTileBytes;
-        const uint32_t d_tmem = tmem + (sbuf ? L::kColS1 : L::kColS0);
+      auto issue_qk = [&](int t, uint32_t k_addr) {
+        const uint32_t q_addr = sq_addr + t * L::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * L::kHalfBytes + (ks & 3) * 32;
-          tc_mma_ss(d_tmem, umma_desc_sw128(sq_addr + koff, 16, 1024),
+          tc_mma_ss(tmem + L::col_s(t), umma_desc_sw128(q_addr + koff, 16, 1024),
                     umma_desc_sw128(k_addr + koff, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[sbuf]);
-        tc_commit(&ring_empty[slot]);
-        if (++slot == kSlots) { slot = 0; phase ^= 1u; }
+        tc_commit(&s_full[t]);
       };
-      auto issue_pv = [&](int sbuf, bool accumulate) {
-        const uint32_t v_addr = ring_addr + slot * L::kTileBytes;
-        const uint32_t a_tmem = tmem + (sbuf ? L::kColS1 : L::kColS0);
+      auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
 #pragma unroll
-        for (int kk = 0; kk < kPfBN / 16; ++kk) {
-          tc_mma_ts(tmem + L::kColO, a_tmem + kk * 8,
+        for (int kk = 0; kk < kPfBN / 16; ++kk)
+          tc_mma_ts(tmem + L::col_o(t), tmem + L::col_s(t) + kk * 8,
                     umma_desc_sw128(v_addr + kk * 2048, L::kHalfBytes, 1024), idesc_pv,
                     (accumulate || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&pv_done[sbuf]);
-        tc_commit(&ring_empty[slot]);
+        tc_commit(&pv_done[t]);
+      };
+      auto next_slot = [&]() {
         if (++slot == kSlots) { slot = 0; phase ^= 1u; }
       };
 
+      // S_A(0), S_B(0)
       if (ok) ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_qk(0);
+        const uint32_t k_addr = ring_addr + slot * L::kTileBytes;
+        issue_qk(0, k_addr);
+        issue_qk(1, k_addr);
+        tc_commit(&ring_empty[slot]);
+        next_slot();
       }
       for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv) {
+        const uint32_t par = (uint32_t)(j & 1);
+        // V_j
+        ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
+        if (!ok) break;
+        const uint32_t v_addr = ring_addr + slot * L::kTileBytes;
+        const int v_slot = slot;
+        next_slot();
+        const bool more = j + 1 < n_kv;
+        uint32_t k_addr = 0;
+        int k_slot = 0;
+        if (more) {
           ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
-          // S buffer (j+1)%2 still holds P_{j-1} until PV_{j-1} completes
-          if (ok && j >= 1)
-            ok = mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &abort_flag);
           if (!ok) break;
-          tc_fence_after();
-          issue_qk((j + 1) & 1);
+          k_addr = ring_addr + slot * L::kTileBytes;
+          k_slot = slot;
+          next_slot();
         }
-        ok = mbar_wait(&p_full[j & 1], (uint32_t)((j >> 1) & 1), &abort_flag);
-        if (ok) ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
+        // tile A: PV_A(j), then S_A(j+1) once PV_A(j) has read P_A(j)
+        ok = mbar_wait(&p_full[0], par, &abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(j & 1, j > 0);
+        issue_pv(0, v_addr, j > 0);
+        if (more) {
+          ok = mbar_wait(&pv_done[0], par, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, k_addr);
+        }
+        // tile B
+        ok = mbar_wait(&p_full[1], par, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, v_addr, j > 0);
+        tc_commit(&ring_empty[v_slot]);
+        if (more) {
+          ok = mbar_wait(&pv_done[1], par, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(1, k_addr);
+          tc_commit(&ring_empty[k_slot]);
+        }
       }
       // every MMA of this thread must finish before tensor memory is freed
       tc_commit(mma_drain);
       mbar_wait(mma_drain, 0, nullptr);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPfRegsSoftmax));
     // ======================================================== softmax
+    const int t = (warp >> 2) - 1;                // query tile of this warpgroup
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // row within the tile
+    const int q0 = q_blk + t * kPfBM;             // first query row of the tile
     const int qi = q0 + r;                        // query index
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_addr = lane_addr + L::col_s(t);
+    const uint32_t o_addr = lane_addr + L::col_o(t);
     const long long row_lim = p.causal ? (long long)qi + off : (long long)1 << 40;
-    float m_ref = -INFINITY;                      // exponent reference (log2 domain)
-    float l_sum = 0.f;      // sum of the bf16-rounded weights that feed P.V (normalises O)
-    float l_exact = 0.f;    // sum of the unrounded weights (gives the LSE)
+    float m_ref = -INFINITY;  // exponent reference (log2 domain)
+    float l_sum = 0.f;        // sum of the bf16-rounded weights that feed P.V (normalises O)
+    float l_exact = 0.f;      // sum of the unrounded weights (gives the LSE)
     bool ok = true;
 
     for (int j = 0; j < n_kv && ok; ++j) {
-      ok = mbar_wait_warp(&s_full[j & 1], (uint32_t)((j >> 1) & 1), &abort_flag);
+      ok = mbar_wait_warp(&s_full[t], (uint32_t)(j & 1), &abort_flag);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_addr = lane_addr + ((j & 1) ? L::kColS1 : L::kColS0);
       float s[kPfBN];
       {
         uint32_t* su = reinterpret_cast<uint32_t*>(s);
@@ -282,18 +322,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         l_exact *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // rescale O (TMEM) once PV_{j-1} has landed
-        ok = mbar_wait_warp(&pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+        // Rescale O_t in TMEM.  PV_t(j-1) has completed: the MMA warp waited
+        // for it before issuing the S_t(j) that this step just read.
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t ov[32];
-          tmem_ld32(lane_addr + L::kColO + c, ov);
+          tmem_ld32(o_addr + c, ov);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(lane_addr + L::kColO + c, ov);
+          tmem_st32(o_addr + c, ov);
         }
       }
       // P = exp2(s * scale_log2 - m_ref), rounded to bf16, written over S
@@ -327,29 +365,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tmem_st32(s_addr + 32, pk + 32);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[t]);
     }
 
     // ---- epilogue
-    if (ok && n_kv > 0)
-      ok = mbar_wait_warp(&pv_done[(n_kv - 1) & 1], (uint32_t)(((n_kv - 1) >> 1) & 1), &abort_flag);
+    if (ok && n_kv > 0) ok = mbar_wait_warp(&pv_done[t], (uint32_t)((n_kv - 1) & 1), &abort_flag);
+    uint8_t* so = sq + t * L::kTileBytes;   // Q_t's slot: every S_t(j) is done with it
     if (ok) {
       tc_fence_after();
       const float inv_l = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-      // O tile -> bf16 -> shared memory (the Q slot, free now) in the
-      // 128-byte swizzled layout of the O tensor map
+      // O tile -> bf16 -> shared memory in the 128-byte swizzled layout of
+      // the O tensor map
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t ov[32];
         if (n_kv > 0) {
-          tmem_ld32(lane_addr + L::kColO + c, ov);
+          tmem_ld32(o_addr + c, ov);
           tc_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
         const int h = c / 64;
-        uint8_t* row_base = sq + h * L::kHalfBytes + r * 128;
+        uint8_t* row_base = so + h * L::kHalfBytes + r * 128;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {          // 4 chunks of 8 columns
           const int chunk = ((c % 64) / 8) + ch;
@@ -371,11 +409,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       fence_proxy_async_smem();
     }
-    // all four softmax warps meet here whatever happened; store only if none gave up
-    const bool stop = bar_sync_or(1, 128, !ok || abort_flag);
-    if (!stop && warp == 2 && lane == 0) {
+    // the four warps of this tile meet here whatever happened; store only if
+    // none of the CTA's warps gave up
+    const bool stop = bar_sync_or(1 + t, 128, !ok || abort_flag);
+    if (!stop && quarter == 0 && lane == 0 && q0 < p.Sq) {
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h) tma_store_3d(&tm_o, sq + h * L::kHalfBytes, h * 64, q0, bh);
+      for (int h = 0; h < kHalves; ++h) tma_store_3d(&tm_o, so + h * L::kHalfBytes, h * 64, q0, bh);
       tma_store_commit();
       tma_store_wait_all();
     }
