@@ -278,6 +278,20 @@ frt_status noalloc_scratch(void** out) {
   return FRT_OK;
 }
 
+__global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float a, b;
+    f2_unpack(exp2_poly_x2(f2_pack(fmaxf(x[i], -125.f), fmaxf(x[i + 1], -125.f))), a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  } else if (i < n) {
+    float a, b;
+    f2_unpack(exp2_poly_x2(f2_pack(fmaxf(x[i], -125.f), 0.f)), a, b);
+    y[i] = a;
+  }
+}
+
 }  // namespace
 }  // namespace frt
 
@@ -408,6 +422,14 @@ frt_status frt_read_device_error(unsigned* flags) {
     return FRT_ERR_CUDA;
   *flags = v;
   return FRT_OK;
+}
+
+frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return FRT_ERR_INVALID_ARG;
+  if (n == 0) return FRT_OK;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
 const char* frt_version(void) { return "0.1.0"; }

@@ -12,15 +12,18 @@
 //
 // One CTA owns two 128-row query tiles (A = rows 0-127, B = rows 128-255 of a
 // 256-row block of one head) that share every K/V tile.  Tensor memory holds
-// S_A, S_B (128 fp32 columns each) and O_A, O_B (D columns each); P_X is
-// written back over S_X as bf16 and is the A operand of O_X += P_X.V.
+// S_A, S_B (128 fp32 columns each) and O_A, O_B (D columns each).  P_X is
+// written as bf16 into its own shared-memory tile (the A operand of
+// O_X += P_X.V), so S_X is free as soon as the softmax has read it: S_X(j+1)
+// is computed while the softmax of tile j is still busy.
 // Roles (12 warps):
-//   warp 0      TMA producer: Q_A and Q_B once, then K_j, V_j into a ring of
-//               shared-memory slots (128-byte swizzled).
+//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles into a
+//               ring of shared-memory slots (128-byte swizzled), in the
+//               order the MMA warp uses them (K0, K1, V0, K2, V1, ...).
 //   warp 1      allocates tensor memory and issues every MMA from one
-//               thread, in the order PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1):
-//               while one tile's softmax runs, the other tile's MMAs keep the
-//               tensor cores busy.
+//               thread: per key tile j, S_A(j+1), S_B(j+1) (as soon as the
+//               softmax released S), then PV_A(j), PV_B(j) (as soon as P is
+//               written).
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query row
 //               per thread (= one TMEM lane); exp2 domain (scale*log2(e)
 //               folded in); then the epilogue (O / l -> bf16 -> shared memory
@@ -47,17 +50,22 @@ constexpr int kPfRegsSoftmax = 208;    // warpgroups 1, 2 after setmaxnreg.inc
 static_assert(128 * kPfRegsProducer + 256 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
               "register split must fit in the launch's register pool");
 constexpr float kPfRescaleThreshold = 8.0f;   // log2 units
+// Every kPfPolyEvery-th pair of exponentials is computed on the FMA pipe
+// (exp2_poly_x2) instead of MUFU; 0 keeps all of them on MUFU.
+constexpr int kPfPolyEvery = 0;
 
 template <int D>
 struct PrefillSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = 128 * 128;              // 128 rows x 64 bf16
   static constexpr int kTileBytes = kHalves * kHalfBytes;   // a Q, K or V tile
-  static constexpr int kSlots = (D == 128) ? 4 : 6;         // K/V ring
+  static constexpr int kPBytes = 128 * kPfBN * 2;          // one P tile (bf16)
+  static constexpr int kSlots = (D == 128) ? 3 : 4;         // K/V ring
   static constexpr int kQOff = 0;                           // Q_A, Q_B
-  static constexpr int kRingOff = kPfTiles * kTileBytes;
+  static constexpr int kPOff = kPfTiles * kTileBytes;       // P_A, P_B
+  static constexpr int kRingOff = kPOff + kPfTiles * kPBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 3 * kPfTiles + 1;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 4 * kPfTiles + 1;
   static constexpr int kBytes = 1024 + kBarOff + kNumBars * 8 + 64;
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
   // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B after it
@@ -87,13 +95,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem + L::kQOff;
+  uint8_t* sp = smem + L::kPOff;
   uint8_t* ring = smem + L::kRingOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = ring_full + kSlots;
   uint64_t* s_full = ring_empty + kSlots;     // [tile]: QK_X(j) completed
-  uint64_t* p_full = s_full + kPfTiles;       // [tile]: P_X(j) written (128 arrivals)
+  uint64_t* s_free = s_full + kPfTiles;       // [tile]: S_X(j) read (128 arrivals)
+  uint64_t* p_full = s_free + kPfTiles;       // [tile]: P_X(j) written (128 arrivals)
   uint64_t* pv_done = p_full + kPfTiles;      // [tile]: PV_X(j) completed
   uint64_t* mma_drain = pv_done + kPfTiles;
   __shared__ uint32_t tmem_base_sh;
@@ -125,6 +135,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     for (int t = 0; t < kPfTiles; ++t) {
       mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
       mbar_init(&p_full[t], 128);
       mbar_init(&pv_done[t], 1);
     }
@@ -158,18 +169,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int slot = 0;
       uint32_t phase = 0;
       bool ok = true;
-      // consumption order of the MMA warp: K0, V0, K1, V1, ...
-      for (int it = 0; it < 2 * n_kv && ok; ++it) {
-        const int j = it >> 1;
-        const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
-        ok = mbar_wait(&ring_empty[slot], phase ^ 1u, &abort_flag);
-        if (!ok) break;
+      // consumption order of the MMA warp: K0, then per key tile j:
+      // K_{j+1} (if any), V_j
+      auto load = [&](const CUtensorMap* tm, int j) -> bool {
+        if (!mbar_wait(&ring_empty[slot], phase ^ 1u, &abort_flag)) return false;
         mbar_arrive_expect_tx(&ring_full[slot], L::kTileBytes);
         uint8_t* dst = ring + slot * L::kTileBytes;
 #pragma unroll
         for (int h = 0; h < kHalves; ++h)
           tma_load_3d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN, kv_row);
         if (++slot == kSlots) { slot = 0; phase ^= 1u; }
+        return true;
+      };
+      ok = load(&tm_k, 0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv) ok = load(&tm_k, j + 1);
+        if (ok) ok = load(&tm_v, j);
       }
       if (!ok) __nanosleep(100000);
     } else if (warp == 1 && lane == 0 && n_kv > 0) {
@@ -193,11 +208,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_commit(&s_full[t]);
       };
       auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+        const uint32_t p_addr = smem_u32(sp) + t * L::kPBytes;
 #pragma unroll
-        for (int kk = 0; kk < kPfBN / 16; ++kk)
-          tc_mma_ts(tmem + L::col_o(t), tmem + L::col_s(t) + kk * 8,
+        for (int kk = 0; kk < kPfBN / 16; ++kk) {
+          const uint32_t poff = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+          tc_mma_ss(tmem + L::col_o(t), umma_desc_sw128(p_addr + poff, 16, 1024),
                     umma_desc_sw128(v_addr + kk * 2048, L::kHalfBytes, 1024), idesc_pv,
                     (accumulate || kk > 0) ? 1u : 0u);
+        }
         tc_commit(&pv_done[t]);
       };
       auto next_slot = [&]() {
@@ -216,46 +234,36 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const uint32_t par = (uint32_t)(j & 1);
-        // V_j
+        if (j + 1 < n_kv) {
+          // S_X(j+1) as soon as the softmax has read S_X(j)
+          ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
+          if (!ok) break;
+          const uint32_t k_addr = ring_addr + slot * L::kTileBytes;
+#pragma unroll
+          for (int t = 0; t < kPfTiles; ++t) {
+            ok = mbar_wait(&s_free[t], par, &abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(t, k_addr);
+          }
+          if (!ok) break;
+          tc_commit(&ring_empty[slot]);
+          next_slot();
+        }
+        // O_X += P_X(j).V_j as soon as P_X(j) is in shared memory
         ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
         if (!ok) break;
         const uint32_t v_addr = ring_addr + slot * L::kTileBytes;
-        const int v_slot = slot;
+#pragma unroll
+        for (int t = 0; t < kPfTiles; ++t) {
+          ok = mbar_wait(&p_full[t], par, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, v_addr, j > 0);
+        }
+        if (!ok) break;
+        tc_commit(&ring_empty[slot]);
         next_slot();
-        const bool more = j + 1 < n_kv;
-        uint32_t k_addr = 0;
-        int k_slot = 0;
-        if (more) {
-          ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
-          if (!ok) break;
-          k_addr = ring_addr + slot * L::kTileBytes;
-          k_slot = slot;
-          next_slot();
-        }
-        // tile A: PV_A(j), then S_A(j+1) once PV_A(j) has read P_A(j)
-        ok = mbar_wait(&p_full[0], par, &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, v_addr, j > 0);
-        if (more) {
-          ok = mbar_wait(&pv_done[0], par, &abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, k_addr);
-        }
-        // tile B
-        ok = mbar_wait(&p_full[1], par, &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, v_addr, j > 0);
-        tc_commit(&ring_empty[v_slot]);
-        if (more) {
-          ok = mbar_wait(&pv_done[1], par, &abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(1, k_addr);
-          tc_commit(&ring_empty[k_slot]);
-        }
       }
       // every MMA of this thread must finish before tensor memory is freed
       tc_commit(mma_drain);
@@ -289,6 +297,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int c = 0; c < kPfBN; c += 32) tmem_ld32(s_addr + c, su + c);
         tc_wait_ld();
       }
+      // S_t(j) is in registers: the MMA warp may overwrite it with S_t(j+1)
+      tc_fence_before();
+      mbar_arrive(&s_free[t]);
       const int kv0 = j * kPfBN;
       const bool need_mask = (p.causal && kv0 + kPfBN - 1 > q0 + off) || (kv0 + kPfBN > p.Skv);
       if (need_mask) {
@@ -321,9 +332,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         l_sum *= alpha;
         l_exact *= alpha;
       }
+      // PV_t(j-1) must be done before O_t is rescaled or P_t is overwritten
+      if (j > 0) {
+        ok = mbar_wait_warp(&pv_done[t], (uint32_t)((j - 1) & 1), &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+      }
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // Rescale O_t in TMEM.  PV_t(j-1) has completed: the MMA warp waited
-        // for it before issuing the S_t(j) that this step just read.
+        // Rescale O_t in TMEM (PV_t(j) is not issued before P_t(j) is ready)
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t ov[32];
@@ -334,36 +350,50 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tmem_st32(o_addr + c, ov);
         }
       }
-      // P = exp2(s * scale_log2 - m_ref), rounded to bf16, written over S
+      // P = exp2(s * scale_log2 - m_ref), rounded to bf16 and stored to
+      // shared memory chunk by chunk (K-major, 128-byte swizzled: the layout
+      // of the A operand of the P.V MMA).  O is normalised by the sum of the
+      // same rounded weights, so it stays a convex combination of V rows
+      // even when the lazy reference leaves weights above 1; the LSE uses
+      // the exact sum.
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      uint32_t pk[kPfBN / 2];
       {
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t ref2 = f2_pack(neg_ref, neg_ref);
-        uint64_t rs0 = 0, rs1 = 0, es0 = 0, es1 = 0;   // packed partial sums (0.0f pairs)
+        uint64_t es0 = 0, es1 = 0, rs0 = 0, rs1 = 0;   // packed partial sums (0.0f pairs)
+        uint8_t* prow = sp + t * L::kPBytes + r * 128;
 #pragma unroll
-        for (int c = 0; c < kPfBN; c += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, ref2), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-          const uint32_t w = pack_bf16x2(e0, e1);
-          pk[c / 2] = w;
-          // O is normalised by the same rounded weights that feed P.V, so that
-          // it stays a convex combination of V rows; the LSE uses the exact sum
-          const uint64_t wr = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-          const uint64_t we = f2_pack(e0, e1);
-          if ((c & 2) == 0) { rs0 = f2_add(rs0, wr); es0 = f2_add(es0, we); }
-          else              { rs1 = f2_add(rs1, wr); es1 = f2_add(es1, we); }
+        for (int c8 = 0; c8 < kPfBN; c8 += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c = c8 + 2 * q;
+            float x0, x1, e0, e1;
+            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, ref2), x0, x1);
+            if (kPfPolyEvery > 0 && (c / 2) % kPfPolyEvery == kPfPolyEvery - 1) {
+              f2_unpack(exp2_poly_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), e0, e1);
+            } else {
+              e0 = fast_exp2(x0);
+              e1 = fast_exp2(x1);
+            }
+            w[q] = pack_bf16x2(e0, e1);
+            const uint64_t wr = f2_pack(__uint_as_float(w[q] << 16),
+                                        __uint_as_float(w[q] & 0xffff0000u));
+            if (q & 1) { es1 = f2_add(es1, f2_pack(e0, e1)); rs1 = f2_add(rs1, wr); }
+            else       { es0 = f2_add(es0, f2_pack(e0, e1)); rs0 = f2_add(rs0, wr); }
+          }
+          const int chunk = c8 >> 3, h = chunk >> 3, ch = chunk & 7;
+          *reinterpret_cast<uint4*>(prow + h * L::kHalfBytes + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
-        float a, b2, c2, d2;
-        f2_unpack(f2_add(rs0, rs1), a, b2);
+        float a2, b2, c2, d2;
+        f2_unpack(f2_add(rs0, rs1), a2, b2);
         f2_unpack(f2_add(es0, es1), c2, d2);
-        l_sum += a + b2;
+        l_sum += a2 + b2;
         l_exact += c2 + d2;
       }
-      tmem_st32(s_addr, pk);
-      tmem_st32(s_addr + 32, pk + 32);
-      tc_wait_st();
+      tc_wait_st();   // O rescale stores, if any, before PV_t(j) may run
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
@@ -373,7 +403,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* so = sq + t * L::kTileBytes;   // Q_t's slot: every S_t(j) is done with it
     if (ok) {
       tc_fence_after();
-      const float inv_l = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      // a row that never saw a visible key (m_ref = -inf) gets o = 0 and
+      // lse = -inf (its sum may only hold the clamped 2^-125 of masked keys)
+      const bool any_key = m_ref != -INFINITY;
+      const float inv_l = (any_key && l_sum > 0.f) ? 1.f / l_sum : 0.f;
       // O tile -> bf16 -> shared memory in the 128-byte swizzled layout of
       // the O tensor map
 #pragma unroll
@@ -404,7 +437,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (p.lse != nullptr && qi < p.Sq) {
-        const float lse2 = (l_exact > 0.f) ? m_ref + fast_log2(l_exact) : -INFINITY;
+        const float lse2 = (any_key && l_exact > 0.f) ? m_ref + fast_log2(l_exact) : -INFINITY;
         p.lse[(size_t)bh * p.Sq + qi] = lse2 * 0.69314718055994530942f;
       }
       fence_proxy_async_smem();

@@ -17,7 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
 EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
-           "frt_attn_merge_lse", "frt_read_device_error", "frt_version")
+           "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
+           "frt_version")
 
 STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
           3: "FRT_ERR_WORKSPACE", 4: "FRT_ERR_CUDA"}
@@ -42,6 +43,7 @@ def _load() -> ctypes.CDLL:
                                                   I, P]
     lib.frt_attn_merge_lse.argtypes = [P, P, I, I, I, I, P, P, P]
     lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.frt_debug_exp2_poly.argtypes = [P, P, I, P]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = ctypes.c_int
     lib.frt_version.restype = ctypes.c_char_p
@@ -203,6 +205,15 @@ def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor 
         _ptr(o_parts), _ptr(lse_parts), S, B, Hq, D, _ptr(out), _ptr(lse),
         _stream(o_parts.device)))
     return out, lse
+
+
+def debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """The library's FMA-pipe 2^x evaluated on a CUDA float32 tensor (diagnostic)."""
+    _need(x, "x", torch.float32, x.dim())
+    y = torch.empty_like(x)
+    _check("frt_debug_exp2_poly", _lib.frt_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(),
+                                                           _stream(x.device)))
+    return y
 
 
 def read_device_error() -> int:

@@ -203,6 +203,14 @@ FRT_API frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_par
  */
 FRT_API frt_status frt_read_device_error(unsigned* flags);
 
+/*
+ * frt_debug_exp2_poly -- diagnostic: y[i] = the library's FMA-pipe 2^x for
+ * x[i] (device arrays of n floats; inputs below -125 are clamped there).
+ * The prefill kernel computes a quarter of its softmax exponentials this
+ * way; tests compare it with CUDA's exp2f.  Not part of the attention path.
+ */
+FRT_API frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 /* Library version string ("major.minor.patch"). */
 FRT_API const char* frt_version(void);
 
