@@ -46,6 +46,34 @@ WORKLOAD = ("llama3-8b causal prefill 4k (B1 Hq32 Hkv8 D128) + paged GQA decode 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def source_sha() -> str:
+    """Hash of the CUDA sources, to tell whether profiled counters still apply."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "flash_attention_tiled_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """Per-call DRAM traffic (bytes per launch) from the committed ncu summary,
+    or {} if the kernels changed since it was taken."""
+    import re
+    path = os.path.join(ROOT, "profiles", "dram_traffic__bench_calls.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return {}
+    m_sha = re.search(r"^source-sha256: (\w+)", text, re.M)
+    m_tr = re.search(r"^traffic_bytes: (.*)$", text, re.M)
+    if not m_sha or not m_tr or m_sha.group(1) != source_sha():
+        return {}
+    return {k: float(v) for k, v in (kv.split("=") for kv in m_tr.group(1).split())}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -329,7 +357,12 @@ def run_ours(args, rank, world, local_rank):
     roof["launches_per_step"] = cnt
     roof["avg_launch_us"] = round(t_ms * 1e3 / cnt, 2)
     roof["peak_source"] = f"{peak_src} (burst figure: each kernel runs < 1 ms)"
-    roof["traffic"] = None
+    tr = profiled_traffic()
+    dom_calls = [n for n in names if kernel_of[n] == dom]
+    roof["traffic"] = (round(sum(tr[n] for n in dom_calls) / len(dom_calls))
+                       if tr and all(n in tr for n in dom_calls) else None)
+    roof["traffic_unit"] = "bytes per launch (ncu dram read + write, profiles/)"
+    roof["algorithmic_bytes_per_launch"] = round(by / cnt)
     roof["share_of_step"] = round(t_ms / sum(v[0] for v in per_kernel.values()), 3)
 
     cpu = None
