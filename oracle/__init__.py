@@ -50,8 +50,11 @@ def _load():
         lib.oracle_attn_decode_paged.argtypes = [P, P, P, P, I, P, I, I, P, P,
                                                  I, I, I, I, D, P]
         lib.oracle_merge_lse.argtypes = [P, P, I, I, I, P, P]
+        lib.oracle_attn_prefill_paged.argtypes = [P, P, P, P, I, P, P, I, I, P, P, I, I, I, I,
+                                                  I, I, D]
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows,
-                  lib.oracle_attn_decode_paged, lib.oracle_merge_lse):
+                  lib.oracle_attn_decode_paged, lib.oracle_merge_lse,
+                  lib.oracle_attn_prefill_paged):
             f.restype = I
         _lib = lib
     return _lib
@@ -129,6 +132,25 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float,
                                           D, float(scale),
                                           None if mask is None else _ptr(mask))
     _check(rc, "attn_decode_paged")
+    return o, lse
+
+
+def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, q_lens, causal: bool,
+                       scale: float):
+    """Chunked prefill over a paged cache: q [B,Hq,max_q,D]; pages [P,Hkv,ps,D];
+    block_table [B,maxp]; seq_lens [B] (context incl. the chunk); q_lens [B].
+    Returns (o [B,Hq,max_q,D], lse [B,Hq,max_q]) fp64; padding rows o=0, lse=-inf."""
+    B, Hq, max_q, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    bt, sl, ql = _i32(block_table), _i32(seq_lens), _i32(q_lens)
+    maxp = bt.shape[1]
+    qa, ka, va = _bits(q), _bits(k_pages), _bits(v_pages)
+    o = np.zeros((B, Hq, max_q, D), np.float64)
+    lse = np.zeros((B, Hq, max_q), np.float64)
+    rc = _load().oracle_attn_prefill_paged(_ptr(qa), _ptr(ka), _ptr(va), _ptr(bt), maxp,
+                                           _ptr(sl), _ptr(ql), ps, P, _ptr(o), _ptr(lse), B, Hq,
+                                           Hkv, max_q, D, int(bool(causal)), float(scale))
+    _check(rc, "attn_prefill_paged")
     return o, lse
 
 

@@ -245,6 +245,70 @@ int oracle_attn_decode_paged(const uint16_t *q, const uint16_t *k_pages,
 }
 
 /*
+ * Chunked prefill over a paged KV cache: sequence b holds seq_lens[b] cached
+ * tokens (the new chunk included) in the paged layout of
+ * oracle_attn_decode_paged, and its last q_lens[b] tokens are the queries.
+ *   q [B][Hq][max_q][D] bf16 bits (rows i >= q_lens[b] are padding)
+ *   o [B][Hq][max_q][D], lse [B][Hq][max_q] fp64; padding rows get o = 0,
+ *   lse = -inf.
+ * The cache is gathered through the block table exactly as for decode, then
+ * the definition applies with Sq = q_lens[b], Skv = seq_lens[b] and the
+ * bottom-right causal mask (query i sees keys j <= i + Skv - Sq) when causal.
+ */
+int oracle_attn_prefill_paged(const uint16_t *q, const uint16_t *k_pages,
+                              const uint16_t *v_pages, const int32_t *block_table,
+                              int max_pages, const int32_t *seq_lens, const int32_t *q_lens,
+                              int page_size, int num_pages, double *o, double *lse, int B,
+                              int Hq, int Hkv, int max_q, int D, int causal, double scale)
+{
+    int rc = check_shape(B, Hq, Hkv, max_q, 0, D, scale);
+    if (rc) return rc;
+    if (page_size <= 0 || num_pages < 0 || max_pages < 0) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        long long len = seq_lens[b];
+        if (len < 0 || (len + page_size - 1) / page_size > max_pages) return ORACLE_ERR_ARG;
+        if (q_lens[b] < 0 || q_lens[b] > max_q) return ORACLE_ERR_ARG;
+        for (long long p = 0; p < (len + page_size - 1) / page_size; ++p) {
+            int32_t phys = block_table[(size_t)b * max_pages + p];
+            if (phys < 0 || phys >= num_pages) return ORACLE_ERR_ARG;
+        }
+    }
+    const int g = Hq / Hkv;
+    for (size_t i = 0; i < (size_t)B * Hq * max_q * D; ++i) o[i] = 0.0;
+    for (size_t i = 0; i < (size_t)B * Hq * max_q; ++i) lse[i] = -INFINITY;
+    for (int b = 0; b < B; ++b) {
+        const int len = seq_lens[b], ql = q_lens[b];
+        const size_t per_head = (size_t)len * D;
+        uint16_t *kc = (uint16_t *)malloc(sizeof(uint16_t) * (per_head * Hkv + 1));
+        uint16_t *vc = (uint16_t *)malloc(sizeof(uint16_t) * (per_head * Hkv + 1));
+        if (!kc || !vc) { free(kc); free(vc); return ORACLE_ERR_MEM; }
+        for (int kvh = 0; kvh < Hkv; ++kvh)
+            for (int t = 0; t < len; ++t) {
+                const int32_t phys = block_table[(size_t)b * max_pages + t / page_size];
+                const size_t src = (((size_t)phys * Hkv + kvh) * page_size + t % page_size) * D;
+                const size_t dst = (size_t)kvh * per_head + (size_t)t * D;
+                memcpy(kc + dst, k_pages + src, sizeof(uint16_t) * D);
+                memcpy(vc + dst, v_pages + src, sizeof(uint16_t) * D);
+            }
+        int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+        for (int h = 0; h < Hq; ++h) {
+            const int kvh = h / g;
+            double *s = (double *)malloc(sizeof(double) * ((size_t)ql * len + 1));
+            if (!s) { failed |= 1; continue; }
+            attend_rows(q + ((size_t)b * Hq + h) * max_q * D, kc + (size_t)kvh * per_head,
+                        vc + (size_t)kvh * per_head, o + ((size_t)b * Hq + h) * max_q * D,
+                        lse + ((size_t)b * Hq + h) * max_q, ql, len, D, causal, scale, 0, ql, s);
+            free(s);
+        }
+        free(kc);
+        free(vc);
+        if (failed) return ORACLE_ERR_MEM;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Merge of partial attention results over disjoint key sets by their
  * log-sum-exp.  If part s attended keys K_s with lse_s = log sum_{j in K_s}
  * exp(s_j) and o_s = sum_{j in K_s} exp(s_j - lse_s) v_j, then over the union

@@ -77,3 +77,35 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float):
                 o[b][h][d] = math.fsum(w * r[d] for w, r in zip(weights, rows)) / den
             lse[b][h] = math.log(den)
     return o, lse
+
+
+def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, q_lens, causal: bool,
+                       scale: float):
+    """q[B][Hq][max_q][D]; pages [P][Hkv][ps][D]; each sequence's last q_lens[b]
+    tokens are the queries, bottom-right causal.  Padding rows: o = 0, lse = -inf."""
+    B, Hq, max_q, D = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv, ps = len(k_pages[0]), len(k_pages[0][0])
+    group = Hq // Hkv
+    o = [[[[0.0] * D for _ in range(max_q)] for _ in range(Hq)] for _ in range(B)]
+    lse = [[[-math.inf] * max_q for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        n, nq = seq_lens[b], q_lens[b]
+        for h in range(Hq):
+            kvh = h // group
+            for i in range(nq):
+                weights, rows = [], []
+                for t in range(n):
+                    if causal and t > i + (n - nq):
+                        continue
+                    page = block_table[b][t // ps]
+                    key = k_pages[page][kvh][t % ps]
+                    s = scale * math.fsum(q[b][h][i][d] * key[d] for d in range(D))
+                    weights.append(math.exp(s))
+                    rows.append(v_pages[page][kvh][t % ps])
+                if not rows:
+                    continue
+                den = math.fsum(weights)
+                for d in range(D):
+                    o[b][h][i][d] = math.fsum(w * r[d] for w, r in zip(weights, rows)) / den
+                lse[b][h][i] = math.log(den)
+    return o, lse

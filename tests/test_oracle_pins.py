@@ -304,3 +304,54 @@ def test_oracle_rejects_bad_shapes():
         oracle.attn_fwd(q, k, k, False, 0.5)      # Hq % Hkv != 0
     with pytest.raises(ValueError):
         oracle.attn_fwd(q, q, q, False, -1.0)     # scale <= 0
+
+
+# ------------------------------------------------- chunked prefill, paged cache
+def _chunk_case(lens, q_lens, Hq, Hkv, D, ps, seed):
+    x = inputs.paged(len(lens), Hq, Hkv, D, seq_lens=lens, page_size=ps, seed=seed)
+    max_q = max(q_lens)
+    q = _rand((len(lens), Hq, max_q, D), seed + 1)
+    return x, q, torch.tensor(q_lens, dtype=torch.int32)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_paged_prefill_matches_brute_force(causal):
+    x, q, ql = _chunk_case([9, 5, 13], [4, 5, 1], 4, 2, 6, 4, 40)
+    o, lse = oracle.attn_prefill_paged(q, x["k_pages"], x["v_pages"], x["block_table"],
+                                       x["seq_lens"], ql, causal, 0.41)
+    ob, lb = brute.attn_prefill_paged(_lists(q), _lists(x["k_pages"]), _lists(x["v_pages"]),
+                                      x["block_table"].tolist(), x["seq_lens"].tolist(),
+                                      ql.tolist(), causal, 0.41)
+    np.testing.assert_allclose(o, np.array(ob), rtol=0, atol=1e-12)
+    lb = np.array(lb)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lb))
+    fin = np.isfinite(lb)
+    np.testing.assert_allclose(lse[fin], lb[fin], atol=1e-12)
+    assert np.isfinite(o).all()
+
+
+def test_paged_prefill_equals_contiguous_on_gathered_cache():
+    ps, D, Hq, Hkv = 4, 8, 4, 2
+    x, q, ql = _chunk_case([14, 7], [6, 7], Hq, Hkv, D, ps, 50)
+    o, lse = oracle.attn_prefill_paged(q, x["k_pages"], x["v_pages"], x["block_table"],
+                                       x["seq_lens"], ql, True, 0.3)
+    for b in range(2):
+        n, nq = int(x["seq_lens"][b]), int(ql[b])
+        pages = x["block_table"][b, : (n + ps - 1) // ps].long()
+        kc = x["k_pages"][pages].permute(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :n]
+        vc = x["v_pages"][pages].permute(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :n]
+        oc, lc = oracle.attn_fwd(q[b:b + 1, :, :nq].contiguous(), kc[None].contiguous(),
+                                 vc[None].contiguous(), True, 0.3)
+        np.testing.assert_array_equal(o[b, :, :nq], oc[0])
+        np.testing.assert_array_equal(lse[b, :, :nq], lc[0])
+        assert np.all(o[b, :, nq:] == 0) and np.all(np.isneginf(lse[b, :, nq:]))
+
+
+def test_paged_prefill_of_one_token_is_decode():
+    x, q, ql = _chunk_case([30, 17, 1], [1, 1, 1], 8, 2, 8, 16, 60)
+    o, lse = oracle.attn_prefill_paged(q, x["k_pages"], x["v_pages"], x["block_table"],
+                                       x["seq_lens"], ql, True, 0.25)
+    od, ld = oracle.attn_decode_paged(q[:, :, 0].contiguous(), x["k_pages"], x["v_pages"],
+                                      x["block_table"], x["seq_lens"], 0.25)
+    np.testing.assert_array_equal(o[:, :, 0], od)
+    np.testing.assert_array_equal(lse[:, :, 0], ld)
