@@ -50,20 +50,31 @@ frt_status device_info(DeviceInfo** out) {
           cudaFuncSetAttribute(decode_splitkv_kernel<64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<64>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(prefill_kernel<128, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrefillSmem<128>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(prefill_kernel<64, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PrefillSmem<64>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(prefill_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PrefillSmem<128>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(prefill_kernel<64, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrefillSmem<64>::kBytes) != cudaSuccess)
         return FRT_ERR_CUDA;
       // The prefill kernel hands registers from its producer warpgroup to
       // its softmax warpgroups (setmaxnreg).  That only works if the launch
       // reserves exactly the pool the split adds up to; otherwise the
       // increase would wait forever, so the kernel is never launched.
-      cudaFuncAttributes fa128, fa64;
-      if (cudaFuncGetAttributes(&fa128, prefill_kernel<128>) != cudaSuccess ||
-          cudaFuncGetAttributes(&fa64, prefill_kernel<64>) != cudaSuccess)
+      cudaFuncAttributes fa[4];
+      if (cudaFuncGetAttributes(&fa[0], prefill_kernel<128, false>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa[1], prefill_kernel<64, false>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa[2], prefill_kernel<128, true>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa[3], prefill_kernel<64, true>) != cudaSuccess)
         return FRT_ERR_CUDA;
-      di.prefill_ok = fa128.numRegs == kPfRegsLaunch && fa64.numRegs == kPfRegsLaunch;
+      di.prefill_ok = true;
+      for (const cudaFuncAttributes& a : fa) di.prefill_ok &= a.numRegs == kPfRegsLaunch;
       di.kernels_configured = true;
     }
   }
@@ -205,31 +216,50 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
-// Tiled tensor-core forward (Sq > 1).
+// Tiled tensor-core forward.  Contiguous K/V [B, Hkv, Skv, D] (paged == null),
+// or chunked prefill over a paged cache (paged != null: Sq is the padded
+// chunk length, lengths per sequence are on the device).
+struct PagedKV {
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const int32_t* q_lens;
+  int max_pages, num_pages;
+};
+
 frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
-                          float scale, cudaStream_t stream) {
+                          float scale, cudaStream_t stream, const PagedKV* paged = nullptr) {
   DeviceInfo* di = nullptr;
   frt_status st = device_info(&di);
   if (st != FRT_OK) return st;
   if (!di->prefill_ok) return FRT_ERR_UNSUPPORTED;
   const int n_blocks = (Sq + kPfRows - 1) / kPfRows;
   if (n_blocks > 65535) return FRT_ERR_UNSUPPORTED;
-  // With Skv == 0 every tile has no key tile to visit (o = 0, lse = -inf);
-  // the K/V maps then only need to be valid descriptors, never read.
-  const void* kb = Skv > 0 ? k : q;
-  const void* vb = Skv > 0 ? v : q;
-  const int skv_map = Skv > 0 ? Skv : 1;
   CUtensorMap tq, tk, tv, to;
   const uint32_t box[3] = {64, (uint32_t)kPfBM, 1};
   const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * Hq};
   const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
-  const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)skv_map,
-                             (uint64_t)(Skv > 0 ? B * Hkv : 1)};
-  const uint64_t kstr[2] = {(uint64_t)D * 2, (uint64_t)skv_map * D * 2};
-  if (!make_tmap(&tq, q, 3, qdims, qstr, box) || !make_tmap(&tk, kb, 3, kdims, kstr, box) ||
-      !make_tmap(&tv, vb, 3, kdims, kstr, box) || !make_tmap(&to, o, 3, qdims, qstr, box))
+  if (!make_tmap(&tq, q, 3, qdims, qstr, box) || !make_tmap(&to, o, 3, qdims, qstr, box))
     return FRT_ERR_CUDA;
+  if (paged == nullptr) {
+    // With Skv == 0 every tile has no key tile to visit (o = 0, lse = -inf);
+    // the K/V maps then only need to be valid descriptors, never read.
+    const void* kb = Skv > 0 ? k : q;
+    const void* vb = Skv > 0 ? v : q;
+    const int skv_map = Skv > 0 ? Skv : 1;
+    const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)skv_map,
+                               (uint64_t)(Skv > 0 ? B * Hkv : 1)};
+    const uint64_t kstr[2] = {(uint64_t)D * 2, (uint64_t)skv_map * D * 2};
+    if (!make_tmap(&tk, kb, 3, kdims, kstr, box) || !make_tmap(&tv, vb, 3, kdims, kstr, box))
+      return FRT_ERR_CUDA;
+  } else {
+    // page pool as rows of D: one 16-row box per page and column half
+    const uint64_t kdims[2] = {(uint64_t)D, (uint64_t)paged->num_pages * Hkv * 16};
+    const uint64_t kstr[1] = {(uint64_t)D * 2};
+    const uint32_t pbox[2] = {64, 16};
+    if (!make_tmap(&tk, k, 2, kdims, kstr, pbox) || !make_tmap(&tv, v, 2, kdims, kstr, pbox))
+      return FRT_ERR_CUDA;
+  }
   PrefillParams p;
   p.lse = lse;
   p.B = B;
@@ -241,11 +271,26 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.causal = causal;
   p.n_blocks = n_blocks;
   p.scale_log2 = scale * kLog2e;
+  p.block_table = paged ? paged->block_table : nullptr;
+  p.seq_lens = paged ? paged->seq_lens : nullptr;
+  p.q_lens = paged ? paged->q_lens : nullptr;
+  p.max_pages = paged ? paged->max_pages : 0;
   const dim3 grid((unsigned)(B * Hq), (unsigned)n_blocks);
-  if (D == 128)
-    prefill_kernel<128><<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
-  else
-    prefill_kernel<64><<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
+  if (paged == nullptr) {
+    if (D == 128)
+      prefill_kernel<128, false>
+          <<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
+    else
+      prefill_kernel<64, false>
+          <<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
+  } else {
+    if (D == 128)
+      prefill_kernel<128, true>
+          <<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
+    else
+      prefill_kernel<64, true>
+          <<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
+  }
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
@@ -359,6 +404,35 @@ frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
                          Hq, Hkv, D, scale, 0, workspace, workspace_bytes, stream);
   }
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream);
+}
+
+frt_status frt_attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                                  const int32_t* block_table, int max_pages_per_seq,
+                                  const int32_t* seq_lens, const int32_t* q_lens, int page_size,
+                                  int num_pages, void* o, float* lse, int B, int Hq, int Hkv,
+                                  int max_q, int D, int causal, float scale,
+                                  cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_q < 0 || num_pages < 0 ||
+      max_pages_per_seq < 0 || (causal != 0 && causal != 1) || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  if (page_size != 16) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31) ||
+      (uint64_t)B * Hq * max_q >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
+  if (B == 0 || max_q == 0) return FRT_OK;
+  if (q == nullptr || o == nullptr || k_pages == nullptr || v_pages == nullptr ||
+      block_table == nullptr || seq_lens == nullptr || q_lens == nullptr ||
+      max_pages_per_seq == 0 || num_pages == 0)
+    return FRT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(k_pages) || !aligned16(v_pages) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(q_lens) & 3u))
+    return FRT_ERR_INVALID_ARG;
+  PagedKV pk{block_table, seq_lens, q_lens, max_pages_per_seq, num_pages};
+  return launch_prefill(q, k_pages, v_pages, o, lse, B, Hq, Hkv, max_q, 0, D, causal, scale,
+                        stream, &pk);
 }
 
 frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_parts, int S, int B,

@@ -65,7 +65,7 @@ struct PrefillSmem {
   static constexpr int kPOff = kPfTiles * kTileBytes;       // P_A, P_B
   static constexpr int kRingOff = kPOff + kPfTiles * kPBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 4 * kPfTiles + 1;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 4 * kPfTiles + 1 + 1;
   static constexpr int kBytes = 1024 + kBarOff + kNumBars * 8 + 64;
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
   // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B after it
@@ -80,9 +80,18 @@ struct PrefillParams {
   float* lse;          // [B, Hq, Sq] or nullptr
   int B, Hq, Hkv, g, Sq, Skv, causal, n_blocks;   // n_blocks = ceil(Sq / 256)
   float scale_log2;
+  // paged K/V (chunked prefill): Sq is the padded chunk length max_q, the
+  // per-sequence chunk and context lengths are read on the device
+  const int32_t* block_table;   // [B, max_pages]
+  const int32_t* seq_lens;      // [B] cached tokens, the chunk included
+  const int32_t* q_lens;        // [B] chunk lengths (<= Sq)
+  int max_pages;
 };
 
-template <int D>
+// kPaged: K and V come from a paged cache ([pages, Hkv, 16, D], 2D tensor
+// maps over its rows) through the block table, and each sequence has its own
+// chunk length q_lens[b] and context length seq_lens[b] (bottom-right causal).
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -106,6 +115,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* p_full = s_free + kPfTiles;       // [tile]: P_X(j) written (128 arrivals)
   uint64_t* pv_done = p_full + kPfTiles;      // [tile]: PV_X(j) completed
   uint64_t* mma_drain = pv_done + kPfTiles;
+  uint64_t* v_tail = mma_drain + 1;           // paged: last V tile's tail rows zeroed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -116,16 +126,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int bh = blockIdx.x;                 // b * Hq + hq
   const int blk = p.causal ? (p.n_blocks - 1 - (int)blockIdx.y) : (int)blockIdx.y;
   const int b = bh / p.Hq, hq = bh % p.Hq;
-  const int kv_row = b * p.Hkv + hq / p.g;   // z coordinate in the K/V maps
+  const int kvh = hq / p.g;
+  const int kv_row = b * p.Hkv + kvh;        // z coordinate in the contiguous K/V maps
   const int q_blk = blk * kPfRows;           // first query row of tile A
-  const int off = p.Skv - p.Sq;              // bottom-right causal alignment
-  const int q_last = min(q_blk + kPfRows - 1, p.Sq - 1);
-  const int n_kv_all = (p.Skv + kPfBN - 1) / kPfBN;
-  int n_kv = n_kv_all;
-  if (p.causal) {
+  // this sequence's chunk (query) length and context (key) length
+  int sq_b = p.Sq, skv_b = p.Skv;
+  if (kPaged) {
+    sq_b = min(max(p.q_lens[b], 0), p.Sq);
+    skv_b = min(max(p.seq_lens[b], 0), p.max_pages * 16);
+  }
+  const int off = skv_b - sq_b;              // bottom-right causal alignment
+  const int q_last = min(q_blk + kPfRows - 1, sq_b - 1);
+  const int n_kv_all = (skv_b + kPfBN - 1) / kPfBN;
+  int n_kv = q_last < q_blk ? 0 : n_kv_all;  // a block wholly in the padding has no work
+  if (p.causal && n_kv > 0) {
     const int lim = q_last + off;            // largest key any row of the block sees
     n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kPfBN + 1);
   }
+  // paged: the last key tile needs its V rows past the sequence end zeroed
+  const bool v_tail_fill = kPaged && n_kv > 0 && n_kv * kPfBN > skv_b;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -140,6 +159,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&pv_done[t], 1);
     }
     mbar_init(mma_drain, 1);
+    mbar_init(v_tail, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -154,30 +174,70 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfRegsProducer));
-    if (warp == 0 && lane == 0 && n_kv > 0) {
+    if (warp == 0 && n_kv > 0) {
       // ================================================= TMA producer
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, kPfTiles * L::kTileBytes);
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        mbar_arrive_expect_tx(q_full, kPfTiles * L::kTileBytes);
 #pragma unroll
-      for (int t = 0; t < kPfTiles; ++t)
+        for (int t = 0; t < kPfTiles; ++t)
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h)
-          tma_load_3d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
-                      q_blk + t * kPfBM, bh);
+          for (int h = 0; h < kHalves; ++h)
+            tma_load_3d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
+                        q_blk + t * kPfBM, bh);
+      }
       int slot = 0;
       uint32_t phase = 0;
       bool ok = true;
       // consumption order of the MMA warp: K0, then per key tile j:
       // K_{j+1} (if any), V_j
       auto load = [&](const CUtensorMap* tm, int j) -> bool {
-        if (!mbar_wait(&ring_empty[slot], phase ^ 1u, &abort_flag)) return false;
-        mbar_arrive_expect_tx(&ring_full[slot], L::kTileBytes);
+        if (!mbar_wait_warp(&ring_empty[slot], phase ^ 1u, &abort_flag)) return false;
         uint8_t* dst = ring + slot * L::kTileBytes;
+        if (!kPaged) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&ring_full[slot], L::kTileBytes);
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h)
-          tma_load_3d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN, kv_row);
+            for (int h = 0; h < kHalves; ++h)
+              tma_load_3d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN,
+                          kv_row);
+          }
+        } else {
+          // eight 16-token pages per key tile, each fetched through the block
+          // table into its 16 rows of the tile (both column halves)
+          const int npg = min(kPfBN / 16, (skv_b + 15) / 16 - j * (kPfBN / 16));
+          int row = 0;
+          if (lane < npg) {
+            const int phys = p.block_table[(size_t)b * p.max_pages + j * (kPfBN / 16) + lane];
+            row = (phys * p.Hkv + kvh) * 16;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&ring_full[slot], npg * kHalves * 16 * 128);
+          __syncwarp();
+          if (lane < npg) {
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h)
+              tma_load_2d(dst + h * L::kHalfBytes + lane * 16 * 128, tm, &ring_full[slot],
+                          h * 64, row);
+          }
+          if (tm == &tm_v && j == n_kv - 1 && v_tail_fill) {
+            // rows past the sequence end may hold anything (NaN); P is 0
+            // there but 0 * NaN is not, so they are zeroed before P.V
+            if (!mbar_wait_warp(&ring_full[slot], phase, &abort_flag)) return false;
+            const int valid = skv_b - j * kPfBN;
+            const int chunks = (kPfBN - valid) * 8 * kHalves;   // 16-byte chunks
+            for (int i = lane; i < chunks; i += 32) {
+              const int h = i / ((kPfBN - valid) * 8);
+              const int rem = i % ((kPfBN - valid) * 8);
+              *reinterpret_cast<uint4*>(dst + h * L::kHalfBytes + (valid + rem / 8) * 128 +
+                                        (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(v_tail);
+          }
+        }
         if (++slot == kSlots) { slot = 0; phase ^= 1u; }
         return true;
       };
@@ -252,6 +312,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         // O_X += P_X(j).V_j as soon as P_X(j) is in shared memory
         ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
+        if (ok && v_tail_fill && j == n_kv - 1) ok = mbar_wait(v_tail, 0, &abort_flag);
         if (!ok) break;
         const uint32_t v_addr = ring_addr + slot * L::kTileBytes;
 #pragma unroll
@@ -301,10 +362,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_before();
       mbar_arrive(&s_free[t]);
       const int kv0 = j * kPfBN;
-      const bool need_mask = (p.causal && kv0 + kPfBN - 1 > q0 + off) || (kv0 + kPfBN > p.Skv);
+      const bool need_mask = (p.causal && kv0 + kPfBN - 1 > q0 + off) || (kv0 + kPfBN > skv_b);
       if (need_mask) {
         long long cmax = row_lim - kv0;
-        const long long tail = (long long)p.Skv - 1 - kv0;
+        const long long tail = (long long)skv_b - 1 - kv0;
         if (tail < cmax) cmax = tail;
 #pragma unroll
         for (int c = 0; c < kPfBN; ++c) s[c] = (c <= cmax) ? s[c] : -INFINITY;
@@ -405,7 +466,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_after();
       // a row that never saw a visible key (m_ref = -inf) gets o = 0 and
       // lse = -inf (its sum may only hold the clamped 2^-125 of masked keys)
-      const bool any_key = m_ref != -INFINITY;
+      // rows of the padding past this sequence's chunk are written as o = 0
+      const bool any_key = m_ref != -INFINITY && qi < sq_b;
       const float inv_l = (any_key && l_sum > 0.f) ? 1.f / l_sum : 0.f;
       // O tile -> bf16 -> shared memory in the 128-byte swizzled layout of
       // the O tensor map
@@ -415,7 +477,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (n_kv > 0) {
           tmem_ld32(o_addr + c, ov);
           tc_wait_ld();
-        } else {
+        }
+        if (n_kv == 0 || !any_key) {   // (padding rows may hold NaN from padded queries)
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
@@ -436,7 +499,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           *reinterpret_cast<uint4*>(row_base + ((chunk ^ (r & 7)) << 4)) = v;
         }
       }
-      if (p.lse != nullptr && qi < p.Sq) {
+      if (p.lse != nullptr && qi < p.Sq) {   // padding rows get -inf
         const float lse2 = (any_key && l_exact > 0.f) ? m_ref + fast_log2(l_exact) : -INFINITY;
         p.lse[(size_t)bh * p.Sq + qi] = lse2 * 0.69314718055994530942f;
       }

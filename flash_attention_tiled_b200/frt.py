@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
 EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
+           "frt_attn_prefill_paged",
            "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
            "frt_version")
 
@@ -42,6 +43,8 @@ def _load() -> ctypes.CDLL:
     lib.frt_attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F,
                                                   I, P]
     lib.frt_attn_merge_lse.argtypes = [P, P, I, I, I, I, P, P, P]
+    lib.frt_attn_prefill_paged.argtypes = [P, P, P, P, I, P, P, I, I, P, P, I, I, I, I, I, I, F,
+                                           P]
     lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.frt_debug_exp2_poly.argtypes = [P, P, I, P]
     for name in EXPORTS[:-1]:
@@ -188,6 +191,33 @@ def attn_decode_paged_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: t
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
         _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale, num_splits,
         _stream(q.device)))
+    return out, lse
+
+
+def attn_prefill_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                       block_table: torch.Tensor, seq_lens: torch.Tensor, q_lens: torch.Tensor,
+                       causal: bool = True, scale: float | None = None,
+                       out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                       return_lse: bool = True):
+    """o, lse = chunked prefill of q [B,Hq,max_q,D] over pages [P,Hkv,16,D]."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(q_lens, "q_lens", torch.int32, 1)
+    B, Hq, max_q, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, max_q), dtype=torch.float32, device=q.device)
+    _check("frt_attn_prefill_paged", _lib.frt_attn_prefill_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), _ptr(q_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, max_q, D,
+        int(causal), scale, _stream(q.device)))
     return out, lse
 
 

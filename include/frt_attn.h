@@ -139,6 +139,39 @@ FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, con
                                  size_t* workspace_bytes, cudaStream_t stream);
 
 /*
+ * frt_attn_prefill_paged -- chunked (or variable-length) prefill over a
+ * paged KV cache: the new tokens of each sequence attend to the sequence's
+ * whole cache, their own keys included ("FlashRT-HF-kernels" page,
+ * "Attention operators": paged attention; the FasterTransformer read-through
+ * (pptc.cn), section 3.1: context phase, requests of different lengths
+ * without padding the keys).  The chunk's K/V must already be in the cache.
+ *
+ *   q           [B, Hq, max_q, D] bf16: sequence b's chunk in rows
+ *               0..q_lens[b]-1 (the rest is padding and is not read for o)
+ *   k_pages,
+ *   v_pages     [num_pages, Hkv, 16, D] bf16 (as frt_attn_decode_paged)
+ *   block_table [B, max_pages_per_seq] int32
+ *   seq_lens    [B] int32, device: cached tokens of sequence b, its chunk
+ *               included (clamped to [0, max_pages_per_seq * 16])
+ *   q_lens      [B] int32, device: chunk length of sequence b (clamped to
+ *               [0, max_q]); the chunk is the last q_lens[b] tokens, so with
+ *               causal = 1 query i sees keys j <= i + seq_lens[b] - q_lens[b]
+ *   o           [B, Hq, max_q, D] bf16; lse [B, Hq, max_q] fp32 or NULL;
+ *               padding rows get o = 0, lse = -inf
+ *   page_size   16
+ * Runs the tiled tensor-core kernel with K/V tiles gathered page by page
+ * through the block table.  Needs no workspace.  Tail slots of a sequence's
+ * last page may hold anything, NaN included.
+ */
+FRT_API frt_status frt_attn_prefill_paged(const void* q, const void* k_pages,
+                                          const void* v_pages, const int32_t* block_table,
+                                          int max_pages_per_seq, const int32_t* seq_lens,
+                                          const int32_t* q_lens, int page_size, int num_pages,
+                                          void* o, float* lse, int B, int Hq, int Hkv,
+                                          int max_q, int D, int causal, float scale,
+                                          cudaStream_t stream);
+
+/*
  * frt_attn_decode_paged_noalloc -- frt_attn_decode_paged for callers that
  * cannot allocate device memory.  No page describes this entry point; it is
  * a convenience of this library.

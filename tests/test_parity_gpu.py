@@ -296,3 +296,50 @@ def test_fma_pipe_exp2_against_cuda_exp2f(frt):
     ref = torch.exp2(x.double())
     rel = ((y.double() - ref).abs() / ref).max().item()
     assert rel <= 1e-4, rel
+
+
+# ------------------------------------------- chunked prefill over a paged cache
+PAGED_PREFILL_CASES = [  # lens (context incl. chunk), q_lens, Hq, Hkv, D, causal
+    ([300], [300], 4, 2, 128, True),                  # whole prompt through pages
+    ([1000, 37, 4096], [200, 37, 129], 8, 2, 128, True),   # chunks after context
+    ([513, 700], [1, 256], 4, 4, 64, True),           # D = 64, a one-token chunk
+    ([900, 130], [300, 130], 4, 1, 128, False),       # non-causal, MQA
+    ([2000], [640], 32, 8, 128, True),
+]
+
+
+@pytest.mark.parametrize("case", PAGED_PREFILL_CASES, ids=str)
+def test_prefill_paged(frt, case):
+    lens, qls, Hq, Hkv, D, causal = case
+    x = inputs.paged(len(lens), Hq, Hkv, D, seq_lens=lens, seed=sum(lens) + Hq)
+    max_q = max(qls)
+    g = torch.Generator().manual_seed(7 + D)
+    q = torch.randn(len(lens), Hq, max_q, D, generator=g).to(torch.bfloat16)
+    for b, n in enumerate(qls):       # the padding rows hold NaN: they must not matter
+        q[b, :, n:] = float("nan")
+    ql = torch.tensor(qls, dtype=torch.int32)
+    d = _dev(x)
+    o, lse = frt.attn_prefill_paged(q.cuda(), d["k_pages"], d["v_pages"], d["block_table"],
+                                    d["seq_lens"], ql.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_prefill_paged(q, x["k_pages"], x["v_pages"], x["block_table"],
+                                               x["seq_lens"], ql, causal, 1 / math.sqrt(D))
+    _compare(o, o_ref, lse, lse_ref, str(case))
+    _no_device_error(frt)
+
+
+def test_prefill_paged_matches_contiguous_bitwise(frt):
+    # the same sequence stored contiguously and in shuffled pages gives the same bits
+    n, Hq, Hkv, D = 1000, 8, 2, 128
+    x = inputs.paged(1, Hq, Hkv, D, seq_lens=[n], seed=77, poison=False)
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, Hq, n, D, generator=g).to(torch.bfloat16).cuda()
+    d = _dev(x)
+    pages = x["block_table"][0, : (n + 15) // 16].long()
+    kc = x["k_pages"][pages].permute(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :n][None].contiguous()
+    vc = x["v_pages"][pages].permute(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :n][None].contiguous()
+    o1, l1 = frt.attn_fwd(q, kc.cuda(), vc.cuda(), causal=True)
+    o2, l2 = frt.attn_prefill_paged(q, d["k_pages"], d["v_pages"], d["block_table"],
+                                    d["seq_lens"], torch.tensor([n], dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
