@@ -68,8 +68,9 @@ struct DecodeSmem {
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // cross-warp combine: one warp's register state in fragment order
-  // (D/8 output tiles x 4 accumulators, then m, l, l_exact for 2 row halves)
-  static constexpr int kFragFloats = (D / 8) * 4 + 6;
+  // (D/16 m-tiles x 2 head tiles x 4 accumulators, then m, l, l_exact for
+  // 2 heads of each head tile), sized for two head tiles
+  static constexpr int kFragFloats = (D / 16) * 2 * 4 + 12;
   static constexpr int kScratchFloats = 2 * kFragFloats * 32;
   static constexpr int kScratchOff = kRingBytes;
   static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
@@ -109,14 +110,15 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t box_base, int row, int c
   return box_base + row * 128 + ((((col >> 3) ^ (row & 7))) << 4);
 }
 
-template <int D>
+// kHT: 8-head tiles per segment (1 when a KV head serves at most 8 query
+// heads, else 2; a segment holds at most 16 query heads).
+template <int D, int kHT>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using L = DecodeSmem<D>;
   constexpr int kStages = L::kStages;
-  constexpr int kKSteps = D / 16;     // MMA K-steps of Q.K^T
-  constexpr int kNTiles = D / 8;      // 8-wide output tiles of P.V
+  constexpr int kKSteps = D / 16;     // MMA K-steps of K.Q^T
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -270,10 +272,14 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   }
 
   // ====================================================== consumers (MMA)
+  // S^T = K.Q^T with a page's 16 tokens as the MMA M dimension and the
+  // segment's query heads as N (8 per head tile), then O^T += V^T.P^T with
+  // the head dimension d as M (16 per m-tile), the heads as N and the page's
+  // tokens as K.  With a GQA group of 8 no MMA row or column is padding.
+  constexpr int kMT = D / 16;            // 16-row m-tiles of d in O^T
   const int cw = warp - 1;               // consumer warp index
-  const int quad = lane >> 2;            // MMA row group: head rows quad, quad+8
-  const int qc = lane & 3;               // column pair within the quad
-  const int t0 = 2 * qc;                 // first token column of this lane in an 8-wide tile
+  const int r8 = lane >> 2;              // fragment row: token (S^T) or d (O^T), and head of B
+  const int qc = lane & 3;               // fragment column pair: heads 2qc, 2qc+1
   const uint32_t ring_u32 = smem_u32(ring);
   constexpr float kLn2 = 0.69314718055994530942f;
 
@@ -289,145 +295,170 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int nh = min(kDecHeadsPerSeg, p.g - hg * kDecHeadsPerSeg);
     const int len = dec_len_of(p, pc.b);
 
-    // Q fragments (A operand, row = head, col = d), rows >= nh are zero
-    uint32_t qa[kKSteps][4];
+    // Q^T fragments (B operand of S^T = K.Q^T): head 8*ht + r8, d pairs
+    uint32_t qb[kHT][kKSteps][2];
     {
       const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)pc.b * p.Hq + h0) * D);
 #pragma unroll
-      for (int ks = 0; ks < kKSteps; ++ks) {
-        const int c0 = ks * 16 + 2 * qc;
-        qa[ks][0] = quad < nh ? q32[(quad * D + c0) / 2] : 0u;
-        qa[ks][1] = quad + 8 < nh ? q32[((quad + 8) * D + c0) / 2] : 0u;
-        qa[ks][2] = quad < nh ? q32[(quad * D + c0 + 8) / 2] : 0u;
-        qa[ks][3] = quad + 8 < nh ? q32[((quad + 8) * D + c0 + 8) / 2] : 0u;
+      for (int ht = 0; ht < kHT; ++ht) {
+        const int head = ht * 8 + r8;
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          qb[ht][ks][0] = head < nh ? q32[(head * D + ks * 16 + 2 * qc) / 2] : 0u;
+          qb[ht][ks][1] = head < nh ? q32[(head * D + ks * 16 + 8 + 2 * qc) / 2] : 0u;
+        }
       }
     }
-    float m_run[2] = {-INFINITY, -INFINITY};   // rows quad, quad+8 (exp2 domain)
-    float l_run[2] = {0.f, 0.f};     // this lane's share of the rounded-weight row sums
-    float le_run[2] = {0.f, 0.f};    // and of the exact-weight row sums (for the LSE)
-    float acc[kNTiles][4];
+    // per lane: heads 2qc, 2qc+1 of each head tile (exp2 domain); the sums
+    // are this lane's share over its tokens
+    float m_run[kHT][2], l_run[kHT][2], le_run[kHT][2];
+    float acc[kMT][kHT][4];
 #pragma unroll
-    for (int t = 0; t < kNTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    for (int ht = 0; ht < kHT; ++ht) {
+      m_run[ht][0] = m_run[ht][1] = -INFINITY;
+      l_run[ht][0] = l_run[ht][1] = le_run[ht][0] = le_run[ht][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) acc[mt][ht][0] = acc[mt][ht][1] = acc[mt][ht][2] = acc[mt][ht][3] = 0.f;
+    }
 
     for (int pb = pc.pg0; pb < pc.pg1; pb += kDecStagePages) {
       ok = mbar_wait_warp(&full_bar[stage], phase, &abort_flag);
       if (!ok) break;
       const int page_a = pb + kDecPagesPerWarp * cw;     // this warp's two pages
-      const int valid_a = page_a < pc.pg1 ? min(kDecPage, len - page_a * kDecPage) : 0;
-      const int valid_b =
-          page_a + 1 < pc.pg1 ? min(kDecPage, len - (page_a + 1) * kDecPage) : 0;
-      if (valid_a > 0) {
-        const bool has_b = valid_b > 0;
-        const uint32_t ka = ring_u32 + stage * L::kStageBytes +
-                            kDecPagesPerWarp * cw * 2 * L::kPageBytes;
-        const uint32_t va = ka + L::kPageBytes;
-        const uint32_t kb = ka + 2 * L::kPageBytes;
-        const uint32_t vb = kb + L::kPageBytes;
-
-        // ---- S = Q.K^T: four 16x8 tiles (tokens 0-7, 8-15 of each page)
-        float s[4][4];
+      int valid[2];
+      valid[0] = page_a < pc.pg1 ? min(kDecPage, len - page_a * kDecPage) : 0;
+      valid[1] = page_a + 1 < pc.pg1 ? min(kDecPage, len - (page_a + 1) * kDecPage) : 0;
+      if (valid[0] > 0) {
+        const int npg = valid[1] > 0 ? 2 : 1;
+        const uint32_t base = ring_u32 + stage * L::kStageBytes +
+                              kDecPagesPerWarp * cw * 2 * L::kPageBytes;
+        // ---- S^T = K.Q^T per page (fragment loads of a page issued first)
+        float sacc[2][kHT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+        for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+          for (int ht = 0; ht < kHT; ++ht) sacc[pg][ht][0] = sacc[pg][ht][1] = sacc[pg][ht][2] = sacc[pg][ht][3] = 0.f;
         {
-          const int mi = lane >> 3, r = lane & 7;
-          const int tok = (mi >> 1) * 8 + r;
+          const int mi = lane >> 3, j = lane & 7;
+          const int tok = (mi & 1) * 8 + j;
 #pragma unroll
-          for (int ks = 0; ks < kKSteps; ++ks) {
-            const int col = ks * 16 + (mi & 1) * 8;
-            const uint32_t off = (col >> 6) * L::kBoxBytes;
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(sw128_addr(ka + off, tok, col & 63), b0, b1, b2, b3);
-            mma_bf16_16816(s[0], qa[ks], b0, b1);
-            mma_bf16_16816(s[1], qa[ks], b2, b3);
-            if (has_b) {
-              ldsm_x4(sw128_addr(kb + off, tok, col & 63), b0, b1, b2, b3);
-              mma_bf16_16816(s[2], qa[ks], b0, b1);
-              mma_bf16_16816(s[3], qa[ks], b2, b3);
-            }
-          }
-        }
-        // ---- scores in the exp2 domain; tokens past the sequence end -> -inf
-        // sc[rh][i]: row quad + 8*rh, token (page a) t0, t0+1, t0+8, t0+9,
-        // (page b) t0, t0+1, t0+8, t0+9
-        float sc[2][8];
+          for (int pg = 0; pg < 2; ++pg) {
+            if (pg < npg) {
+              const uint32_t kbase = base + pg * 2 * L::kPageBytes;
+              uint32_t kf[kKSteps][4];
 #pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int tok = t0 + (i & 1) + (i >> 1) * 8;
-            sc[rh][i] = (tok < valid_a) ? s[i >> 1][2 * rh + (i & 1)] * p.scale_log2 : -INFINITY;
-            sc[rh][4 + i] =
-                (tok < valid_b) ? s[2 + (i >> 1)][2 * rh + (i & 1)] * p.scale_log2 : -INFINITY;
-          }
-        }
-        uint32_t pa[4], pbv[4];   // P fragments of page a and page b
-        float alpha[2];
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-          float mx = fmaxf(fmaxf(fmaxf(sc[rh][0], sc[rh][1]), fmaxf(sc[rh][2], sc[rh][3])),
-                           fmaxf(fmaxf(sc[rh][4], sc[rh][5]), fmaxf(sc[rh][6], sc[rh][7])));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float m_new = fmaxf(m_run[rh], mx);
-          alpha[rh] = fast_exp2(m_run[rh] - m_new);   // 0 on the first step
-          m_run[rh] = m_new;
-          float e[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) e[i] = fast_exp2(sc[rh][i] - m_new);
-          const uint32_t w0 = pack_bf16x2(e[0], e[1]), w1 = pack_bf16x2(e[2], e[3]);
-          const uint32_t w2 = pack_bf16x2(e[4], e[5]), w3 = pack_bf16x2(e[6], e[7]);
-          // O is normalised by the bf16-rounded weights that feed P.V; the LSE
-          // uses the exact ones
-          const float psum = (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u)) +
-                             (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u)) +
-                             (__uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xffff0000u)) +
-                             (__uint_as_float(w3 << 16) + __uint_as_float(w3 & 0xffff0000u));
-          const float esum = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-          l_run[rh] = l_run[rh] * alpha[rh] + psum;
-          le_run[rh] = le_run[rh] * alpha[rh] + esum;
-          pa[rh] = w0;        // a0a1 (rh=0) / a2a3 (rh=1): tokens t0, t0+1
-          pa[2 + rh] = w1;    // a4a5 / a6a7: tokens t0+8, t0+9
-          pbv[rh] = w2;
-          pbv[2 + rh] = w3;
-        }
-        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-          for (int t = 0; t < kNTiles; ++t) {
-            acc[t][0] *= alpha[0];
-            acc[t][1] *= alpha[0];
-            acc[t][2] *= alpha[1];
-            acc[t][3] *= alpha[1];
-          }
-        }
-        // ---- O += P.V: V^T fragments by transposing ldmatrix
-        {
-          const int mi = lane >> 3, r = lane & 7;
-          const int tok = (mi & 1) * 8 + r;
-          const bool tail_a = valid_a < kDecPage, tail_b = has_b && valid_b < kDecPage;
-#pragma unroll
-          for (int nt = 0; nt < kNTiles; nt += 2) {
-            const int col = (nt + (mi >> 1)) * 8;
-            const uint32_t off = (col >> 6) * L::kBoxBytes;
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(sw128_addr(va + off, tok, col & 63), b0, b1, b2, b3);
-            if (tail_a) {   // tokens past the sequence end may hold anything (NaN)
-              b0 = (t0 < valid_a ? (b0 & 0xffffu) : 0u) | (t0 + 1 < valid_a ? (b0 & 0xffff0000u) : 0u);
-              b2 = (t0 < valid_a ? (b2 & 0xffffu) : 0u) | (t0 + 1 < valid_a ? (b2 & 0xffff0000u) : 0u);
-              b1 = (t0 + 8 < valid_a ? (b1 & 0xffffu) : 0u) | (t0 + 9 < valid_a ? (b1 & 0xffff0000u) : 0u);
-              b3 = (t0 + 8 < valid_a ? (b3 & 0xffffu) : 0u) | (t0 + 9 < valid_a ? (b3 & 0xffff0000u) : 0u);
-            }
-            mma_bf16_16816(acc[nt], pa, b0, b1);
-            mma_bf16_16816(acc[nt + 1], pa, b2, b3);
-            if (has_b) {
-              ldsm_x4_trans(sw128_addr(vb + off, tok, col & 63), b0, b1, b2, b3);
-              if (tail_b) {
-                b0 = (t0 < valid_b ? (b0 & 0xffffu) : 0u) | (t0 + 1 < valid_b ? (b0 & 0xffff0000u) : 0u);
-                b2 = (t0 < valid_b ? (b2 & 0xffffu) : 0u) | (t0 + 1 < valid_b ? (b2 & 0xffff0000u) : 0u);
-                b1 = (t0 + 8 < valid_b ? (b1 & 0xffffu) : 0u) | (t0 + 9 < valid_b ? (b1 & 0xffff0000u) : 0u);
-                b3 = (t0 + 8 < valid_b ? (b3 & 0xffffu) : 0u) | (t0 + 9 < valid_b ? (b3 & 0xffff0000u) : 0u);
+              for (int ks = 0; ks < kKSteps; ++ks) {
+                const int col = ks * 16 + (mi >> 1) * 8;
+                ldsm_x4(sw128_addr(kbase + (col >> 6) * L::kBoxBytes, tok, col & 63), kf[ks][0],
+                        kf[ks][1], kf[ks][2], kf[ks][3]);
               }
-              mma_bf16_16816(acc[nt], pbv, b0, b1);
-              mma_bf16_16816(acc[nt + 1], pbv, b2, b3);
+#pragma unroll
+              for (int ks = 0; ks < kKSteps; ++ks)
+#pragma unroll
+                for (int ht = 0; ht < kHT; ++ht)
+                  mma_bf16_16816(sacc[pg][ht], kf[ks], qb[ht][ks][0], qb[ht][ks][1]);
+            }
+          }
+        }
+        // ---- online softmax per head over this step's tokens; tokens past
+        // the sequence end -> -inf.  sc[pg][ht][i]: i = e (token r8, head 2qc+e)
+        // and 2+e (token r8+8)
+        uint32_t pbf[2][kHT][2];   // P^T fragments (B operand) per page and head tile
+        float alpha[kHT][2];
+#pragma unroll
+        for (int ht = 0; ht < kHT; ++ht) {
+          float sc[2][4];
+#pragma unroll
+          for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int tok = r8 + (i >> 1) * 8;
+              sc[pg][i] = tok < valid[pg] ? sacc[pg][ht][i] * p.scale_log2 : -INFINITY;
+            }
+          float e[2][4];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float mx = fmaxf(fmaxf(sc[0][hh], sc[0][2 + hh]), fmaxf(sc[1][hh], sc[1][2 + hh]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float m_new = fmaxf(m_run[ht][hh], mx);
+            alpha[ht][hh] = fast_exp2(m_run[ht][hh] - m_new);   // 0 on the first step
+            m_run[ht][hh] = m_new;
+#pragma unroll
+            for (int pg = 0; pg < 2; ++pg) {
+              e[pg][hh] = fast_exp2(sc[pg][hh] - m_new);
+              e[pg][2 + hh] = fast_exp2(sc[pg][2 + hh] - m_new);
+            }
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            l_run[ht][hh] *= alpha[ht][hh];
+            le_run[ht][hh] *= alpha[ht][hh];
+          }
+#pragma unroll
+          for (int pg = 0; pg < 2; ++pg) {
+            // rows r8 (lo) and r8+8 (hi) of S^T as bf16 pairs (heads 2qc, 2qc+1)
+            const uint32_t lo = pack_bf16x2(e[pg][0], e[pg][1]);
+            const uint32_t hi = pack_bf16x2(e[pg][2], e[pg][3]);
+            // O is normalised by the bf16-rounded weights that feed P.V; the
+            // LSE uses the exact ones
+            l_run[ht][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
+            l_run[ht][1] += __uint_as_float(lo & 0xffff0000u) + __uint_as_float(hi & 0xffff0000u);
+            le_run[ht][0] += e[pg][0] + e[pg][2];
+            le_run[ht][1] += e[pg][1] + e[pg][3];
+            // transpose to the B layout of P^T (token pairs, head r8)
+            pbf[pg][ht][0] = movmatrix_trans(lo);
+            pbf[pg][ht][1] = movmatrix_trans(hi);
+          }
+        }
+        bool any_scale = false;
+#pragma unroll
+        for (int ht = 0; ht < kHT; ++ht) any_scale |= (alpha[ht][0] != 1.f) || (alpha[ht][1] != 1.f);
+        if (__any_sync(0xffffffffu, any_scale)) {
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+            for (int ht = 0; ht < kHT; ++ht) {
+              acc[mt][ht][0] *= alpha[ht][0];
+              acc[mt][ht][1] *= alpha[ht][1];
+              acc[mt][ht][2] *= alpha[ht][0];
+              acc[mt][ht][3] *= alpha[ht][1];
+            }
+        }
+        // ---- O^T += V^T.P^T per page: V^T fragments by transposing ldmatrix
+        {
+          const int mi = lane >> 3, j = lane & 7;
+          const int tok = (mi >> 1) * 8 + j;
+#pragma unroll
+          for (int pg = 0; pg < 2; ++pg) {
+            if (pg < npg) {
+              const uint32_t vbase = base + pg * 2 * L::kPageBytes + L::kPageBytes;
+              uint32_t vf[kMT][4];
+#pragma unroll
+              for (int mt = 0; mt < kMT; ++mt) {
+                const int col = mt * 16 + (mi & 1) * 8;
+                ldsm_x4_trans(sw128_addr(vbase + (col >> 6) * L::kBoxBytes, tok, col & 63),
+                              vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+              }
+              const int v = valid[pg];
+              if (v < kDecPage) {   // tokens past the sequence end may hold anything (NaN)
+                const int t0 = 2 * qc;
+                const uint32_t m01 = (t0 < v ? 0xffffu : 0u) | (t0 + 1 < v ? 0xffff0000u : 0u);
+                const uint32_t m89 = (t0 + 8 < v ? 0xffffu : 0u) | (t0 + 9 < v ? 0xffff0000u : 0u);
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                  vf[mt][0] &= m01;
+                  vf[mt][1] &= m01;
+                  vf[mt][2] &= m89;
+                  vf[mt][3] &= m89;
+                }
+              }
+#pragma unroll
+              for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+                for (int ht = 0; ht < kHT; ++ht)
+                  mma_bf16_16816(acc[mt][ht], vf[mt], pbf[pg][ht][0], pbf[pg][ht][1]);
             }
           }
         }
@@ -440,42 +471,52 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // ---- combine the four warps' states in registers: 2,3 -> 0,1 -> 0
     // stop together if any warp gave up (every consumer gets the same answer)
     if (bar_sync_or(1, kDecWarps * 32, !ok || abort_flag)) break;
+    constexpr int kAccF = kMT * kHT * 4;
 #pragma unroll
     for (int level = 0; level < 2; ++level) {
       const int senders = level == 0 ? 2 : 1;        // warps [senders, 2*senders) send
       if (cw >= senders && cw < 2 * senders) {
         float* dst = scratch + (cw - senders) * L::kFragFloats * 32 + lane;
 #pragma unroll
-        for (int t = 0; t < kNTiles; ++t)
+        for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[(t * 4 + i) * 32] = acc[t][i];
+          for (int ht = 0; ht < kHT; ++ht)
 #pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-          dst[(kNTiles * 4 + rh) * 32] = m_run[rh];
-          dst[(kNTiles * 4 + 2 + rh) * 32] = l_run[rh];
-          dst[(kNTiles * 4 + 4 + rh) * 32] = le_run[rh];
-        }
+            for (int i = 0; i < 4; ++i) dst[((mt * kHT + ht) * 4 + i) * 32] = acc[mt][ht][i];
+#pragma unroll
+        for (int ht = 0; ht < kHT; ++ht)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            dst[(kAccF + ht * 6 + hh) * 32] = m_run[ht][hh];
+            dst[(kAccF + ht * 6 + 2 + hh) * 32] = l_run[ht][hh];
+            dst[(kAccF + ht * 6 + 4 + hh) * 32] = le_run[ht][hh];
+          }
       }
       asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
       if (cw < senders) {
         const float* src = scratch + cw * L::kFragFloats * 32 + lane;
-        float wa[2], wb[2];
+        float wa[kHT][2], wb[kHT][2];
 #pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-          const float mo = src[(kNTiles * 4 + rh) * 32];
-          const float mn = fmaxf(m_run[rh], mo);
-          // a state that saw no key has m = -inf and contributes nothing
-          wa[rh] = (m_run[rh] == -INFINITY) ? 0.f : fast_exp2(m_run[rh] - mn);
-          wb[rh] = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
-          m_run[rh] = mn;
-          l_run[rh] = l_run[rh] * wa[rh] + src[(kNTiles * 4 + 2 + rh) * 32] * wb[rh];
-          le_run[rh] = le_run[rh] * wa[rh] + src[(kNTiles * 4 + 4 + rh) * 32] * wb[rh];
-        }
+        for (int ht = 0; ht < kHT; ++ht)
 #pragma unroll
-        for (int t = 0; t < kNTiles; ++t)
+          for (int hh = 0; hh < 2; ++hh) {
+            const float mo = src[(kAccF + ht * 6 + hh) * 32];
+            const float mn = fmaxf(m_run[ht][hh], mo);
+            // a state that saw no key has m = -inf and contributes nothing
+            wa[ht][hh] = (m_run[ht][hh] == -INFINITY) ? 0.f : fast_exp2(m_run[ht][hh] - mn);
+            wb[ht][hh] = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+            m_run[ht][hh] = mn;
+            l_run[ht][hh] = l_run[ht][hh] * wa[ht][hh] + src[(kAccF + ht * 6 + 2 + hh) * 32] * wb[ht][hh];
+            le_run[ht][hh] = le_run[ht][hh] * wa[ht][hh] + src[(kAccF + ht * 6 + 4 + hh) * 32] * wb[ht][hh];
+          }
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            acc[t][i] = acc[t][i] * wa[i >> 1] + src[(t * 4 + i) * 32] * wb[i >> 1];
+        for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+          for (int ht = 0; ht < kHT; ++ht)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              acc[mt][ht][i] = acc[mt][ht][i] * wa[ht][i & 1] +
+                               src[((mt * kHT + ht) * 4 + i) * 32] * wb[ht][i & 1];
       }
       asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
     }
@@ -486,33 +527,39 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int slot = c + seg;
     if (cw == 0) {
 #pragma unroll
-      for (int rh = 0; rh < 2; ++rh) {
-        float ls = l_run[rh], le = le_run[rh];
-        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-        le += __shfl_xor_sync(0xffffffffu, le, 1);
-        le += __shfl_xor_sync(0xffffffffu, le, 2);
-        const int r = quad + 8 * rh;
-        if (r < nh) {
-          const float inv = 1.f / ls;
-          const float lse2 = m_run[rh] + fast_log2(le);
-          if (whole) {
-            __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D;
+      for (int ht = 0; ht < kHT; ++ht)
 #pragma unroll
-            for (int t = 0; t < kNTiles; ++t)
-              *reinterpret_cast<uint32_t*>(orow + t * 8 + t0) =
-                  pack_bf16x2(acc[t][2 * rh] * inv, acc[t][2 * rh + 1] * inv);
-            if (qc == 0 && p.lse != nullptr) p.lse[(size_t)pc.b * p.Hq + h0 + r] = lse2 * kLn2;
-          } else {
-            float* orow = p.ws_o + ((size_t)slot * kDecHeadsPerSeg + r) * D;
+        for (int hh = 0; hh < 2; ++hh) {
+          // each head's sums are spread over the 8 lanes with the same qc
+          float ls = l_run[ht][hh], le = le_run[ht][hh];
 #pragma unroll
-            for (int t = 0; t < kNTiles; ++t)
-              *reinterpret_cast<float2*>(orow + t * 8 + t0) =
-                  make_float2(acc[t][2 * rh] * inv, acc[t][2 * rh + 1] * inv);
-            if (qc == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
+          for (int off = 4; off < 32; off <<= 1) {
+            ls += __shfl_xor_sync(0xffffffffu, ls, off);
+            le += __shfl_xor_sync(0xffffffffu, le, off);
+          }
+          const int r = ht * 8 + 2 * qc + hh;   // head within the segment
+          if (r < nh) {
+            const float inv = 1.f / ls;
+            const float lse2 = m_run[ht][hh] + fast_log2(le);
+            if (whole) {
+              __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D;
+#pragma unroll
+              for (int mt = 0; mt < kMT; ++mt) {
+                orow[mt * 16 + r8] = __float2bfloat16(acc[mt][ht][hh] * inv);
+                orow[mt * 16 + 8 + r8] = __float2bfloat16(acc[mt][ht][2 + hh] * inv);
+              }
+              if (r8 == 0 && p.lse != nullptr) p.lse[(size_t)pc.b * p.Hq + h0 + r] = lse2 * kLn2;
+            } else {
+              float* orow = p.ws_o + ((size_t)slot * kDecHeadsPerSeg + r) * D;
+#pragma unroll
+              for (int mt = 0; mt < kMT; ++mt) {
+                orow[mt * 16 + r8] = acc[mt][ht][hh] * inv;
+                orow[mt * 16 + 8 + r8] = acc[mt][ht][2 + hh] * inv;
+              }
+              if (r8 == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
+            }
           }
         }
-      }
       if (!whole) {
         // ticket: the last piece of this segment to finish merges all of them
         __threadfence();

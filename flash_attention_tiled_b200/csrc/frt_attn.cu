@@ -44,10 +44,16 @@ frt_status device_info(DeviceInfo** out) {
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FRT_ERR_CUDA;
       di.sm_count = sms;
-      if (cudaFuncSetAttribute(decode_splitkv_kernel<128>,
+      if (cudaFuncSetAttribute(decode_splitkv_kernel<128, 1>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<128>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(decode_splitkv_kernel<64>,
+          cudaFuncSetAttribute(decode_splitkv_kernel<128, 2>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<128>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(decode_splitkv_kernel<64, 1>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<64>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(decode_splitkv_kernel<64, 2>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<64>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(prefill_kernel<128, false>,
@@ -209,10 +215,19 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
   p.ws_count = reinterpret_cast<unsigned*>(ws + wl.count_off);
 
-  if (D == 128)
-    decode_splitkv_kernel<128><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
-  else
-    decode_splitkv_kernel<64><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
+  // one 8-head tile per segment when a KV head serves at most 8 query heads
+  const bool one_tile = g <= 8;
+  if (D == 128) {
+    if (one_tile)
+      decode_splitkv_kernel<128, 1><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
+    else
+      decode_splitkv_kernel<128, 2><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
+  } else {
+    if (one_tile)
+      decode_splitkv_kernel<64, 1><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
+    else
+      decode_splitkv_kernel<64, 2><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
+  }
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
