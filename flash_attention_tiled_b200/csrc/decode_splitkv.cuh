@@ -16,20 +16,22 @@
 // grid take equal contiguous shares of that line, so every CTA streams the
 // same number of pages whatever the length mix.  The piece of a segment that
 // falls inside one CTA is reduced to one partial (o, lse); a segment wholly
-// inside one CTA is written out directly, otherwise the last CTA to finish
-// one of its pieces merges all of them by log-sum-exp (an atomic ticket per
-// segment; no CTA ever waits for another).
+// inside one CTA is written out directly.  The partials of split segments
+// are combined by log-sum-exp in a second, small kernel (decode_merge_kernel)
+// that spreads every (sequence, query head) row over its own CTA; it is
+// launched as a programmatic dependent, so it is resident and waiting when
+// the streaming kernel ends.  No CTA ever waits for another.
 //
-// Inside a CTA: warp 0 streams pages into a ring of shared-memory stages with
-// TMA (one 128-byte swizzled box per page and matrix, one mbarrier per
-// stage), looking pages
-// up in the block table; warps 1..W each take two pages (32 tokens) of every
-// stage and compute S = Q.K^T and O += P.V with warp-level bf16 MMAs in which
-// the segment's query heads form the M dimension, so each K/V page is read
-// from HBM once for all heads of its group.  Scores live in the exp2 domain
-// (scale * log2(e) folded in); the online max/sum use quad shuffles.  At the
-// end of a piece the warps' states are combined in registers (two levels
-// through shared memory) and written by one warp.
+// Inside a CTA (two per SM): warp 0 streams pages into a ring of
+// shared-memory stages with TMA (one 128-byte swizzled box per page and
+// matrix, one mbarrier per stage), looking pages up in the block table;
+// warps 1..W each take two pages (32 tokens) of every stage and compute
+// S^T = K.Q^T and O^T += V^T.P^T with warp-level bf16 MMAs in which a page's
+// tokens form the M dimension of the first and the segment's query heads the
+// N dimension of both, so each K/V page is read from HBM once for all heads
+// of its group.  Scores live in the exp2 domain (scale * log2(e) folded in).
+// At the end of a piece the warps' states are combined in registers (through
+// shared memory) and written by one warp.
 #pragma once
 
 #include "frt_device.cuh"
@@ -37,10 +39,13 @@
 namespace frt {
 
 constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
-constexpr int kDecWarps = 4;          // consumer warps per CTA
+constexpr int kDecWarps = 2;          // consumer warps per CTA (a power of two)
 constexpr int kDecPagesPerWarp = 2;   // pages a consumer warp takes per stage
 constexpr int kDecStagePages = kDecWarps * kDecPagesPerWarp;
 constexpr int kDecThreads = 32 * (kDecWarps + 1);
+// Two CTAs share an SM: two independent TMA rings per SM keep more page
+// copies in flight than one ring twice as deep.
+constexpr int kDecCtasPerSm = 2;
 constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
 constexpr int kDecMaxBatch = 1024;    // prefix table held in shared memory
 
@@ -53,10 +58,12 @@ struct DecodeParams {
   int max_pages;                 // paged: block-table row length
   int contig_len;                // contiguous: keys per sequence (Skv)
   int B, Hq, Hkv, g, hgroups;    // g = Hq / Hkv, hgroups = ceil(g / 16)
+  int parts;                     // CTAs of the streaming kernel's grid
   float scale_log2;              // scale * log2(e)
   float* ws_o;                   // [slots, 16, D] fp32 partial outputs (normalised)
   float* ws_lse;                 // [slots, 16] fp32 partial LSE (log2 domain)
-  unsigned* ws_count;            // [segments] arrival tickets, zero between calls
+  int2* ws_seg;                  // [segments] CTAs holding its pieces {first, last};
+                                 // {-1, -1}: written out whole (or empty)
 };
 
 template <int D>
@@ -64,20 +71,22 @@ struct DecodeSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 64 bf16
   static constexpr int kPageBytes = kHalves * kBoxBytes;              // K or V of one page
-  static constexpr int kStageBytes = kDecStagePages * 2 * kPageBytes; // K+V of 8 pages
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kStageBytes = kDecStagePages * 2 * kPageBytes; // K+V of 4 pages
+  static constexpr int kStages = (D == 128) ? 3 : 6;                  // 96 KB ring
   static constexpr int kRingBytes = kStages * kStageBytes;
   // cross-warp combine: one warp's register state in fragment order
   // (D/16 m-tiles x 2 head tiles x 4 accumulators, then m, l, l_exact for
   // 2 heads of each head tile), sized for two head tiles
   static constexpr int kFragFloats = (D / 16) * 2 * 4 + 12;
-  static constexpr int kScratchFloats = 2 * kFragFloats * 32;
+  static constexpr int kScratchFloats = (kDecWarps / 2) * kFragFloats * 32;
   static constexpr int kScratchOff = kRingBytes;
   static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
   static constexpr int kBarOff = kPrefixOff + ((kDecMaxBatch + 1) * 4 + 15) / 16 * 16;
   static constexpr int kBytes = 1024 /*alignment slack*/ + kBarOff + 2 * kStages * 8;
   static_assert(kBarOff % 8 == 0, "mbarriers need 8-byte alignment");
-  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+  // per SM: 228 KB, of which each CTA also reserves 1 KB (static shared
+  // variables live in the slack below)
+  static_assert(kDecCtasPerSm * (kBytes + 1024 + 64) <= 228 * 1024, "shared memory budget");
 };
 
 // Pages of sequence b (seq_len clamped to [0, max_pages * 16]).
@@ -113,7 +122,7 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t box_base, int row, int c
 // kHT: 8-head tiles per segment (1 when a KV head serves at most 8 query
 // heads, else 2; a segment holds at most 16 query heads).
 template <int D, int kHT>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using L = DecodeSmem<D>;
@@ -129,11 +138,16 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* empty_bar = full_bar + kStages;
   __shared__ int abort_flag;
-  __shared__ int s_is_last;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int nseg_b = p.Hkv * p.hgroups;   // segments per sequence
+
+  // Inputs may come from the kernel before this one in the stream: wait for
+  // it (a no-op unless launched as a programmatic dependent), then let the
+  // merge kernel that follows get resident.
+  griddep_wait();
+  griddep_launch_dependents();
 
   // ---- per-sequence page prefix (warp 0: chunked scan), barriers
   if (warp == 0) {
@@ -178,6 +192,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
       p.o[(size_t)b * p.Hq * D + i] = __float2bfloat16(0.f);
     if (p.lse != nullptr)
       for (int i = threadIdx.x; i < p.Hq; i += blockDim.x) p.lse[(size_t)b * p.Hq + i] = -INFINITY;
+    for (int i = threadIdx.x; i < nseg_b; i += blockDim.x) p.ws_seg[(size_t)b * nseg_b + i] = make_int2(-1, -1);
   }
   if (c >= C) return;
 
@@ -468,13 +483,13 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
       if (++stage == kStages) { stage = 0; phase ^= 1u; }
     }
 
-    // ---- combine the four warps' states in registers: 2,3 -> 0,1 -> 0
+    // ---- combine the warps' states in registers, halving the number of
+    // holders each level (warps [n/2, n) send to [0, n/2))
     // stop together if any warp gave up (every consumer gets the same answer)
     if (bar_sync_or(1, kDecWarps * 32, !ok || abort_flag)) break;
     constexpr int kAccF = kMT * kHT * 4;
 #pragma unroll
-    for (int level = 0; level < 2; ++level) {
-      const int senders = level == 0 ? 2 : 1;        // warps [senders, 2*senders) send
+    for (int senders = kDecWarps / 2; senders >= 1; senders >>= 1) {
       if (cw >= senders && cw < 2 * senders) {
         float* dst = scratch + (cw - senders) * L::kFragFloats * 32 + lane;
 #pragma unroll
@@ -560,65 +575,111 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
           }
         }
-      if (!whole) {
-        // ticket: the last piece of this segment to finish merges all of them
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          const int c_first = dec_cta_of(pc.seg_u0, T, C);
-          const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C);
-          const unsigned parts = (unsigned)(c_last - c_first + 1);
-          const unsigned prev = atomicAdd(&p.ws_count[seg], 1u);
-          if (prev == parts - 1) {
-            p.ws_count[seg] = 0u;   // ready for the next call
-            __threadfence();
-            last = c_first + 1;
-          }
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (lane == 0) s_is_last = last;
-      }
+      // the owner of the segment's first page records where its pieces are
+      if (pc.pg0 == 0 && lane == 0)
+        p.ws_seg[seg] = whole ? make_int2(-1, -1) : make_int2(c, dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C));
     }
-    if (!whole) {
-      asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
-      if (s_is_last) {
-        // single pass over the parts with a running maximum; every thread
-        // owns 4 consecutive d of one row, loads of later parts overlap
-        const int c_first = s_is_last - 1;
-        const int c_last = dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C);
-        const int ct = threadIdx.x - 32;
-        for (int e = ct; e < nh * (D / 4); e += kDecWarps * 32) {
-          const int r = e / (D / 4), d4 = (e % (D / 4)) * 4;
-          float M = -INFINITY, S = 0.f;
-          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-          for (int cc = c_first; cc <= c_last; ++cc) {
-            const size_t sl = (size_t)(cc + seg);
-            const float x = __ldcg(&p.ws_lse[sl * kDecHeadsPerSeg + r]);
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                &p.ws_o[(sl * kDecHeadsPerSeg + r) * D + d4]));
-            const float mn = fmaxf(M, x);
-            const float a = fast_exp2(M - mn);   // 0 while M = -inf
-            const float w = fast_exp2(x - mn);
-            S = S * a + w;
-            o4.x = o4.x * a + w * v.x;
-            o4.y = o4.y * a + w * v.y;
-            o4.z = o4.z * a + w * v.z;
-            o4.w = o4.w * a + w * v.w;
-            M = mn;
-          }
-          const float inv = 1.f / S;
-          __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D + d4;
-          *reinterpret_cast<uint2*>(orow) =
-              make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
-          if (d4 == 0 && p.lse != nullptr)
-            p.lse[(size_t)pc.b * p.Hq + h0 + r] = (M + fast_log2(S)) * kLn2;
-        }
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch, s_is_last reuse
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch reuse
   } while (next_piece(pc));
+}
+
+// Log-sum-exp merge of split segments' partials: o = sum_c 2^(lse_c - M) o_c /
+// sum_c 2^(lse_c - M), lse = M + log2 of that denominator, over the CTAs c that
+// held a piece of the segment (M = max lse_c).  Rows are (sequence, query
+// head); CTA x takes rows x, x + grid, ... and first finds, in parallel,
+// which of them belong to split segments.  Inside a row the parts are spread
+// over kGroups thread groups (one float4 of the row per thread) and the groups'
+// sums are added through shared memory.
+constexpr int kMergeThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const DecodeParams p) {
+  constexpr int kV = D / 4;                    // float4 per row
+  constexpr int kGroups = kMergeThreads / kV;  // part groups
+  constexpr float kLn2 = 0.69314718055994530942f;
+  __shared__ float4 red[kGroups][kV];
+  __shared__ float red_s[kGroups];
+  __shared__ float red_m[kMergeThreads / 32];
+  __shared__ int list[kMergeThreads];
+  __shared__ int nlist;
+  griddep_wait();   // the streaming kernel's partials and segment table
+
+  const int t = threadIdx.x, grp = t / kV, l = t % kV;
+  const int nseg_b = p.Hkv * p.hgroups;
+  const long long rows = (long long)p.B * p.Hq;
+  auto seg_of = [&](int row, int& r) {
+    const int b = row / p.Hq, h = row % p.Hq;
+    const int kvh = h / p.g, hq = h % p.g;
+    r = hq % kDecHeadsPerSeg;
+    return b * nseg_b + kvh * p.hgroups + hq / kDecHeadsPerSeg;
+  };
+  for (long long base = 0; blockIdx.x + base * gridDim.x < rows; base += kMergeThreads) {
+    if (t == 0) nlist = 0;
+    __syncthreads();
+    const long long row = blockIdx.x + (base + t) * gridDim.x;
+    if (row < rows) {
+      int r;
+      const int seg = seg_of((int)row, r);
+      // (a range outside this grid can only be left over from a call that
+      // stopped on a device error; it is skipped so no read leaves the slots)
+      const int2 info = p.ws_seg[seg];
+      if (info.x >= 0 && info.x <= info.y && info.y < p.parts) list[atomicAdd(&nlist, 1)] = (int)row;
+    }
+    __syncthreads();
+    const int n = nlist;
+    for (int k = 0; k < n; ++k) {
+      const int row_k = list[k];
+      int r;
+      const int seg = seg_of(row_k, r);
+      const int2 info = p.ws_seg[seg];
+      // M = max over the parts' LSEs (every part holds at least one key)
+      float m = -INFINITY;
+      for (int cc = info.x + t; cc <= info.y; cc += kMergeThreads)
+        m = fmaxf(m, p.ws_lse[(size_t)(cc + seg) * kDecHeadsPerSeg + r]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (t % 32 == 0) red_m[t / 32] = m;
+      __syncthreads();
+      float M = red_m[0];
+#pragma unroll
+      for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, red_m[w]);
+      // this group's parts
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float S = 0.f;
+#pragma unroll 4
+      for (int cc = info.x + grp; cc <= info.y; cc += kGroups) {
+        const size_t sl = (size_t)(cc + seg) * kDecHeadsPerSeg + r;
+        const float w = fast_exp2(p.ws_lse[sl] - M);
+        const float4 v = reinterpret_cast<const float4*>(p.ws_o + sl * D)[l];
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
+        S += w;
+      }
+      red[grp][l] = acc;
+      if (l == 0) red_s[grp] = S;
+      __syncthreads();
+      if (t < kV) {
+        float4 o4 = red[0][t];
+        float St = red_s[0];
+#pragma unroll
+        for (int g2 = 1; g2 < kGroups; ++g2) {
+          const float4 v = red[g2][t];
+          o4.x += v.x;
+          o4.y += v.y;
+          o4.z += v.z;
+          o4.w += v.w;
+          St += red_s[g2];
+        }
+        const float inv = 1.f / St;
+        *reinterpret_cast<uint2*>(p.o + (size_t)row_k * D + 4 * t) =
+            make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
+        if (t == 0 && p.lse != nullptr) p.lse[row_k] = (M + fast_log2(St)) * kLn2;
+      }
+      __syncthreads();   // red, red_m reuse
+    }
+  }
 }
 
 }  // namespace frt

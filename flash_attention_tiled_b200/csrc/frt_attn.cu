@@ -2,6 +2,7 @@
 // argument validation, work planning, TMA descriptor encoding and kernel
 // launches on the caller's stream.  This is the library's single translation
 // unit; the kernels live in the .cuh files it includes.
+#include <algorithm>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -135,17 +136,18 @@ bool scale_ok(float scale) { return scale > 0.f && isfinite(scale); }
 
 // ---------------------------------------------------- decode workspace
 struct DecodeWorkspace {
-  size_t o_off, lse_off, count_off, total;
+  size_t o_off, lse_off, seg_off, total;
 };
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Counters first: their offset does not depend on the problem shape.
+// [segments] piece ranges, [slots, 16] partial LSEs, [slots, 16, D] partial
+// outputs; every call writes what it later reads, so nothing carries over.
 DecodeWorkspace decode_ws_layout(long long parts, long long segments, int D) {
   DecodeWorkspace w;
   const long long slots = parts + segments;
-  w.count_off = 0;
-  w.lse_off = round_up((size_t)segments * sizeof(unsigned), 256);
+  w.seg_off = 0;
+  w.lse_off = round_up((size_t)segments * sizeof(int2), 256);
   w.o_off = w.lse_off + round_up((size_t)slots * kDecHeadsPerSeg * sizeof(float), 256);
   w.total = w.o_off + round_up((size_t)slots * kDecHeadsPerSeg * D * sizeof(float), 256);
   return w;
@@ -172,7 +174,7 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       frt_status st = device_info(&di);
       if (st != FRT_OK) return st;
     }
-    parts = di->sm_count;
+    parts = kDecCtasPerSm * di->sm_count;
   }
   const DecodeWorkspace wl = decode_ws_layout(parts, segments, D);
   if (query) {
@@ -209,11 +211,12 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
   p.Hkv = Hkv;
   p.g = g;
   p.hgroups = hgroups;
+  p.parts = parts;
   p.scale_log2 = scale * kLog2e;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
-  p.ws_count = reinterpret_cast<unsigned*>(ws + wl.count_off);
+  p.ws_seg = reinterpret_cast<int2*>(ws + wl.seg_off);
 
   // one 8-head tile per segment when a KV head serves at most 8 query heads
   const bool one_tile = g <= 8;
@@ -228,7 +231,26 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
     else
       decode_splitkv_kernel<64, 2><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
   }
-  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return FRT_ERR_CUDA;
+
+  // The merge of split segments, as a programmatic dependent of the kernel
+  // above: its CTAs are scheduled while that one still runs and start when
+  // it has finished.  One CTA per row, up to eight per SM.
+  const long long rows = (long long)B * Hq;
+  const unsigned merge_grid = (unsigned)std::min<long long>(rows, 8ll * di->sm_count);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(merge_grid);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err = (D == 128) ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<128>, p)
+                                     : cudaLaunchKernelEx(&cfg, decode_merge_kernel<64>, p);
+  return err == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
 // Tiled tensor-core forward.  Contiguous K/V [B, Hkv, Skv, D] (paged == null),
@@ -490,13 +512,8 @@ frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pages,
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != FRT_OK) return st;
-  // The scratch keeps whatever the previous call left there; the arrival
-  // counters at its start must read zero when the kernel begins.
-  const int g = Hkv > 0 ? Hq / Hkv : 0;
-  const size_t counter_bytes =
-      (size_t)B * Hkv * ((g + kDecHeadsPerSeg - 1) / kDecHeadsPerSeg) * sizeof(unsigned);
-  if (counter_bytes > 0 && cudaMemsetAsync(scratch, 0, counter_bytes, stream) != cudaSuccess)
-    return FRT_ERR_CUDA;
+  // The kernels write every word of the scratch they read later in the
+  // call, so whatever a previous call left there is harmless.
   size_t have = kNoAllocScratchBytes;
   return frt_attn_decode_paged(q, k_pages, v_pages, block_table, max_pages_per_seq, seq_lens,
                                page_size, num_pages, o, lse, B, Hq, Hkv, D, scale, num_splits,

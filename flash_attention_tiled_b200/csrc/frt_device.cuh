@@ -196,6 +196,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
       : "memory");
 }
 
+// Programmatic dependent launch.  griddep_wait blocks until the grids this
+// one depends on have finished and their writes are visible (returns at once
+// for an ordinary launch); griddep_launch_dependents lets the next grid in the
+// stream, when launched as a programmatic dependent, be scheduled early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Transpose of an 8x8 matrix of 16-bit values held one pair per thread in
 // the MMA fragment layout (row lane/4, columns 2*(lane%4), +1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {

@@ -431,7 +431,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int c = c8 + 2 * q;
             float x0, x1, e0, e1;
             f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, ref2), x0, x1);
-            if (kPfPolyEvery > 0 && (c / 2) % kPfPolyEvery == kPfPolyEvery - 1) {
+            constexpr int kEvery = kPfPolyEvery > 0 ? kPfPolyEvery : 1;
+            if (kPfPolyEvery > 0 && (c / 2) % kEvery == kEvery - 1) {
               f2_unpack(exp2_poly_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), e0, e1);
             } else {
               e0 = fast_exp2(x0);

@@ -88,9 +88,9 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be contiguous")
 
 
-# Zero-filled workspaces, one per (device, stream, shape): the library's
-# arrival counters return to zero after every call, so a workspace can be
-# reused by later calls of the same shape ordered on the same stream.
+# Workspaces, one per (device, stream, shape): a call writes every word of
+# the workspace it later reads, so one buffer serves all later calls of the
+# same shape ordered on the same stream.
 _workspaces: dict = {}
 
 

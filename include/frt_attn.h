@@ -111,21 +111,23 @@ FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, voi
  *               negative one is read as 0
  *   o           [B, Hq, D] bf16;  lse [B, Hq] fp32, may be NULL
  *   page_size   16 in this version
- *   num_splits  number of work partitions the cache is cut into (0 = one
+ *   num_splits  number of work partitions the cache is cut into (0 = two
  *               per SM, the default); every partition streams an equal
  *               share of all sequences' pages, so mixed lengths balance
  *   workspace   device scratch of *workspace_bytes bytes, 16-byte aligned.
  *               Size query: a call with q == NULL only writes the required
  *               size to *workspace_bytes and returns FRT_OK.  The size
- *               depends on B, Hq, Hkv, D and num_splits only.  It holds
- *               arrival counters that must read zero when a call starts:
- *               zero-fill a workspace before its first use; every call
- *               leaves the counters at zero again, so later calls with the
- *               same shape may reuse it as is.  A workspace last used for a
- *               different shape (or a call that reported a device error)
- *               must be zero-filled again first.  Calls that share a
- *               workspace must be ordered on the device (the same stream,
- *               or events).
+ *               depends on B, Hq, Hkv, D and num_splits only.  Its
+ *               contents need no preparation: each call writes every word
+ *               it later reads, so a workspace may be reused for any call
+ *               it is large enough for.  Calls that share a workspace must
+ *               be ordered on the device (the same stream, or events).
+ *
+ * Two kernels run on `stream`: the streaming kernel, then a small merge of
+ * the partitions' partial results, launched as its programmatic dependent
+ * (it is scheduled early and waits on the device for the first to finish).
+ * Both start by waiting for the work before them in the stream, so the call
+ * is ordered like any other stream operation.
  *
  * Block-table entries outside [0, num_pages) read zeros (the copy engine's
  * bounds), never out-of-bounds memory.  Tail slots of the last page of a
@@ -189,13 +191,11 @@ FRT_API frt_status frt_attn_prefill_paged(const void* q, const void* k_pages,
  * (held until the process exits).  It allocates nothing and frees nothing.
  *   - Limit: a problem whose workspace (see frt_attn_decode_paged's size
  *     query) exceeds 16 MiB is rejected with FRT_ERR_WORKSPACE before
- *     anything runs.  At D = 128 with one partition per SM that is roughly
- *     B * Hkv <= 1800 (fewer when a KV head serves more than 16 query heads).
+ *     anything runs.  At D = 128 with two partitions per SM that is roughly
+ *     B * Hkv <= 1700 (fewer when a KV head serves more than 16 query heads).
  *   - The first call made with a given device current looks up that
  *     device's buffer address; make that first call before any stream
  *     capture on that device.
- *   - Each call first clears the buffer's arrival counters on `stream`
- *     (a memset of B * Hkv * ceil(Hq/Hkv/16) * 4 bytes), then launches.
  *   - All calls on a device share the one buffer, and it keeps what the
  *     last call left in it: calls that can overlap on the device (different
  *     streams without ordering) race and corrupt each other's results.

@@ -85,8 +85,9 @@ def test_decode_workspace_query_with_explicit_splits():
     rc = frt.lib().frt_attn_decode_paged(NULL, NULL, NULL, NULL, 8, NULL, 16, 10, NULL, NULL, 2,
                                          64, 8, 128, 0.1, 37, NULL, ctypes.byref(need), NULL)
     assert rc == 0
-    # partials for 37 + 16 slots of 16 rows x 128 fp32, LSEs and 16 counters
-    assert need.value >= (37 + 16) * 16 * 128 * 4 + (37 + 16) * 16 * 4 + 16 * 4
+    # partials for 37 + 16 slots of 16 rows x 128 fp32, their LSEs and a
+    # piece range (two int32) per segment
+    assert need.value >= (37 + 16) * 16 * 128 * 4 + (37 + 16) * 16 * 4 + 16 * 8
 
 
 @pytest.mark.parametrize("S,B,Hq,D,code", [(0, 1, 1, 64, 1), (1, -1, 1, 64, 1), (2, 1, 0, 64, 1),
