@@ -175,6 +175,9 @@ class Step:
     """The four calls of one step, with inputs resident on the device."""
 
     ALL = ("prefill", "paged", "long", "contig")
+    # kernels each call launches: prefill_kernel; decode_splitkv_kernel then
+    # decode_merge_kernel
+    LAUNCHES = {"prefill": 1, "paged": 2, "long": 2, "contig": 2}
 
     def __init__(self, device, names=ALL):
         from flash_attention_tiled_b200 import frt
@@ -253,20 +256,30 @@ def run_ours(args, rank, world, local_rank):
             st.call(n)
     # Per-call timing graphs: R x (L2 flush, call) and R x (L2 flush) alone;
     # a call's device time is the difference divided by R, so neither the
-    # graph launch nor the flush is counted.
+    # graph launch nor the flush is counted.  The flush writes a buffer of
+    # twice the L2 size, then reads another one: the write evicts the call's
+    # inputs, the read evicts the written lines, so their write-back to HBM
+    # happens inside the flush and is not charged to the call.
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+    flush_w = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+    flush_r = torch.ones(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=device)
+    flush_acc = torch.empty((), dtype=torch.float32, device=device)
+
+    def flush():
+        flush_w.fill_(1.0)
+        torch.sum(flush_r, dim=0, out=flush_acc)
+
     R = 20
     g_flush = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_flush, stream=stream):
         for _ in range(R):
-            flush.fill_(1.0)
+            flush()
     g_call = {}
     for n in names:
         g_call[n] = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_call[n], stream=stream):
             for _ in range(R):
-                flush.fill_(1.0)
+                flush()
                 st.call(n)
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -336,7 +349,9 @@ def run_ours(args, rank, world, local_rank):
             rec["frac"] = round(rec["gbs"] / peaks["hbm_gbs"], 4)
         calls[n] = rec
     # The dominant kernel is the one with the largest share of a step: the
-    # decode kernel serves three calls, the prefill kernel one.
+    # decode kernel serves three calls, the prefill kernel one.  A decode
+    # call's time also holds its small merge kernel (timed together, so the
+    # streaming kernel's fraction is if anything understated).
     kernel_of = {"prefill": "prefill_kernel<128>", "paged": "decode_splitkv_kernel<128>",
                  "long": "decode_splitkv_kernel<128>", "contig": "decode_splitkv_kernel<128>"}
     per_kernel = {}
@@ -388,12 +403,13 @@ def run_ours(args, rank, world, local_rank):
                              "graph of 20 flushes, divided by 20",
                    "l2": "step working set ~0.9 GB > 126 MB L2 and every call's inputs are "
                          "evicted by the calls before it; per-call timings flush L2 "
-                         "(2x L2 size written) before each call"},
+                         "before each call (2x L2 size written, then another 2x L2 "
+                         "read so the written lines are clean)"},
         "calls": calls,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": len(names) * args.steps,
+        "gpu_launches": sum(Step.LAUNCHES[n] for n in names) * args.steps,
         "clocks": sampler.summary(),
     }
     return line

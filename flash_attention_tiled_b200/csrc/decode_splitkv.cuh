@@ -587,22 +587,23 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // sum_c 2^(lse_c - M), lse = M + log2 of that denominator, over the CTAs c that
 // held a piece of the segment (M = max lse_c).  Rows are (sequence, query
 // head); CTA x takes rows x, x + grid, ... and first finds, in parallel,
-// which of them belong to split segments.  Inside a row the parts are spread
-// over kGroups thread groups (one float4 of the row per thread) and the groups'
-// sums are added through shared memory.
-constexpr int kMergeThreads = 256;
+// which of them belong to split segments.  Inside a row the parts are dealt
+// round-robin to kGroups thread groups (one float4 of the row per thread),
+// each reducing its parts in one pass with a running maximum; the groups'
+// states are then combined through shared memory.
+constexpr int kMergeThreads = 1024;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const DecodeParams p) {
   constexpr int kV = D / 4;                    // float4 per row
-  constexpr int kGroups = kMergeThreads / kV;  // part groups
+  constexpr int kGroups = kMergeThreads / kV;  // part groups (32 at D = 128)
   constexpr float kLn2 = 0.69314718055994530942f;
   __shared__ float4 red[kGroups][kV];
-  __shared__ float red_s[kGroups];
-  __shared__ float red_m[kMergeThreads / 32];
+  __shared__ float red_m[kGroups], red_s[kGroups];
   __shared__ int list[kMergeThreads];
   __shared__ int nlist;
   griddep_wait();   // the streaming kernel's partials and segment table
+  griddep_launch_dependents();
 
   const int t = threadIdx.x, grp = t / kV, l = t % kV;
   const int nseg_b = p.Hkv * p.hgroups;
@@ -632,52 +633,54 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
       int r;
       const int seg = seg_of(row_k, r);
       const int2 info = p.ws_seg[seg];
-      // M = max over the parts' LSEs (every part holds at least one key)
-      float m = -INFINITY;
-      for (int cc = info.x + t; cc <= info.y; cc += kMergeThreads)
-        m = fmaxf(m, p.ws_lse[(size_t)(cc + seg) * kDecHeadsPerSeg + r]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (t % 32 == 0) red_m[t / 32] = m;
-      __syncthreads();
-      float M = red_m[0];
-#pragma unroll
-      for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, red_m[w]);
-      // this group's parts
+      // this group's parts, one pass with a running maximum (every part
+      // holds at least one key, so its LSE is finite)
+      float m = -INFINITY, S = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float S = 0.f;
 #pragma unroll 4
       for (int cc = info.x + grp; cc <= info.y; cc += kGroups) {
         const size_t sl = (size_t)(cc + seg) * kDecHeadsPerSeg + r;
-        const float w = fast_exp2(p.ws_lse[sl] - M);
+        const float x = p.ws_lse[sl];
         const float4 v = reinterpret_cast<const float4*>(p.ws_o + sl * D)[l];
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
-        S += w;
+        const float mn = fmaxf(m, x);
+        const float a = fast_exp2(m - mn);   // 0 while m = -inf
+        const float w = fast_exp2(x - mn);
+        S = S * a + w;
+        acc.x = acc.x * a + w * v.x;
+        acc.y = acc.y * a + w * v.y;
+        acc.z = acc.z * a + w * v.z;
+        acc.w = acc.w * a + w * v.w;
+        m = mn;
       }
       red[grp][l] = acc;
-      if (l == 0) red_s[grp] = S;
+      if (l == 0) {
+        red_m[grp] = m;
+        red_s[grp] = S;
+      }
       __syncthreads();
       if (t < kV) {
-        float4 o4 = red[0][t];
-        float St = red_s[0];
+        float M = -INFINITY;
 #pragma unroll
-        for (int g2 = 1; g2 < kGroups; ++g2) {
+        for (int g2 = 0; g2 < kGroups; ++g2) M = fmaxf(M, red_m[g2]);
+        float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float St = 0.f;
+#pragma unroll 8
+        for (int g2 = 0; g2 < kGroups; ++g2) {
+          const float mg = red_m[g2];
+          const float w = mg == -INFINITY ? 0.f : fast_exp2(mg - M);   // a group with no part
           const float4 v = red[g2][t];
-          o4.x += v.x;
-          o4.y += v.y;
-          o4.z += v.z;
-          o4.w += v.w;
-          St += red_s[g2];
+          o4.x += w * v.x;
+          o4.y += w * v.y;
+          o4.z += w * v.z;
+          o4.w += w * v.w;
+          St += w * red_s[g2];
         }
         const float inv = 1.f / St;
         *reinterpret_cast<uint2*>(p.o + (size_t)row_k * D + 4 * t) =
             make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
         if (t == 0 && p.lse != nullptr) p.lse[row_k] = (M + fast_log2(St)) * kLn2;
       }
-      __syncthreads();   // red, red_m reuse
+      __syncthreads();   // red, red_m, red_s reuse
     }
   }
 }

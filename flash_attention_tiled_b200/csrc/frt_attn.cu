@@ -3,6 +3,7 @@
 // launches on the caller's stream.  This is the library's single translation
 // unit; the kernels live in the .cuh files it includes.
 #include <algorithm>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -141,6 +142,26 @@ struct DecodeWorkspace {
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Every kernel is launched as a programmatic dependent of the work before it
+// in the stream: it is scheduled while that work still runs, and its first
+// instruction (griddepcontrol.wait) holds it until that work has finished
+// and its writes are visible, so ordering is the same as a plain launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // [segments] piece ranges, [slots, 16] partial LSEs, [slots, 16, D] partial
 // outputs; every call writes what it later reads, so nothing carries over.
 DecodeWorkspace decode_ws_layout(long long parts, long long segments, int D) {
@@ -220,36 +241,20 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
 
   // one 8-head tile per segment when a KV head serves at most 8 query heads
   const bool one_tile = g <= 8;
-  if (D == 128) {
-    if (one_tile)
-      decode_splitkv_kernel<128, 1><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
-    else
-      decode_splitkv_kernel<128, 2><<<parts, kDecThreads, DecodeSmem<128>::kBytes, stream>>>(tk, tv, p);
-  } else {
-    if (one_tile)
-      decode_splitkv_kernel<64, 1><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
-    else
-      decode_splitkv_kernel<64, 2><<<parts, kDecThreads, DecodeSmem<64>::kBytes, stream>>>(tk, tv, p);
-  }
-  if (cudaGetLastError() != cudaSuccess) return FRT_ERR_CUDA;
+  const size_t smem = (D == 128) ? DecodeSmem<128>::kBytes : DecodeSmem<64>::kBytes;
+  auto* kernel = (D == 128) ? (one_tile ? decode_splitkv_kernel<128, 1> : decode_splitkv_kernel<128, 2>)
+                            : (one_tile ? decode_splitkv_kernel<64, 1> : decode_splitkv_kernel<64, 2>);
+  if (launch_pdl(kernel, dim3(parts), dim3(kDecThreads), smem, stream, tk, tv, p) != cudaSuccess)
+    return FRT_ERR_CUDA;
 
-  // The merge of split segments, as a programmatic dependent of the kernel
-  // above: its CTAs are scheduled while that one still runs and start when
-  // it has finished.  One CTA per row, up to eight per SM.
+  // The merge of split segments: its CTAs are scheduled while the kernel
+  // above still runs and start when it has finished.  One CTA per row, up to
+  // two per SM.
   const long long rows = (long long)B * Hq;
-  const unsigned merge_grid = (unsigned)std::min<long long>(rows, 8ll * di->sm_count);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(merge_grid);
-  cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t err = (D == 128) ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<128>, p)
-                                     : cudaLaunchKernelEx(&cfg, decode_merge_kernel<64>, p);
+  const unsigned merge_grid = (unsigned)std::min<long long>(rows, 2ll * di->sm_count);
+  const cudaError_t err =
+      launch_pdl((D == 128) ? decode_merge_kernel<128> : decode_merge_kernel<64>, dim3(merge_grid),
+                 dim3(kMergeThreads), 0, stream, p);
   return err == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
@@ -313,22 +318,13 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.q_lens = paged ? paged->q_lens : nullptr;
   p.max_pages = paged ? paged->max_pages : 0;
   const dim3 grid((unsigned)(B * Hq), (unsigned)n_blocks);
-  if (paged == nullptr) {
-    if (D == 128)
-      prefill_kernel<128, false>
-          <<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
-    else
-      prefill_kernel<64, false>
-          <<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
-  } else {
-    if (D == 128)
-      prefill_kernel<128, true>
-          <<<grid, kPfThreads, PrefillSmem<128>::kBytes, stream>>>(tq, tk, tv, to, p);
-    else
-      prefill_kernel<64, true>
-          <<<grid, kPfThreads, PrefillSmem<64>::kBytes, stream>>>(tq, tk, tv, to, p);
-  }
-  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+  auto* kernel = (paged == nullptr)
+                     ? (D == 128 ? prefill_kernel<128, false> : prefill_kernel<64, false>)
+                     : (D == 128 ? prefill_kernel<128, true> : prefill_kernel<64, true>);
+  const size_t smem = (D == 128) ? PrefillSmem<128>::kBytes : PrefillSmem<64>::kBytes;
+  return launch_pdl(kernel, grid, dim3(kPfThreads), smem, stream, tq, tk, tv, to, p) == cudaSuccess
+             ? FRT_OK
+             : FRT_ERR_CUDA;
 }
 
 // ------------------------------------------- decode without caller scratch
@@ -484,13 +480,11 @@ frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_parts, int 
     return FRT_ERR_INVALID_ARG;
   const long long blocks = (rows + kMergeWarps - 1) / kMergeWarps;
   if (blocks > 0x7fffffffLL) return FRT_ERR_UNSUPPORTED;
-  if (D == 128)
-    merge_lse_kernel<128><<<(unsigned)blocks, kMergeWarps * 32, 0, stream>>>(
-        o_parts, lse_parts, S, rows, static_cast<__nv_bfloat16*>(o), lse);
-  else
-    merge_lse_kernel<64><<<(unsigned)blocks, kMergeWarps * 32, 0, stream>>>(
-        o_parts, lse_parts, S, rows, static_cast<__nv_bfloat16*>(o), lse);
-  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+  return launch_pdl(D == 128 ? merge_lse_kernel<128> : merge_lse_kernel<64>, dim3((unsigned)blocks),
+                    dim3(kMergeWarps * 32), 0, stream, o_parts, lse_parts, S, rows,
+                    static_cast<__nv_bfloat16*>(o), lse) == cudaSuccess
+             ? FRT_OK
+             : FRT_ERR_CUDA;
 }
 
 frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pages,

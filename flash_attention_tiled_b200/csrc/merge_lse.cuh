@@ -24,6 +24,8 @@ merge_lse_kernel(const float* __restrict__ o_parts, const float* __restrict__ ls
   constexpr int kPer = D / 32;   // elements per lane (2 or 4)
   const long long row = (long long)blockIdx.x * kMergeWarps + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  griddep_wait();   // the parts may come from the kernel before this one
+  griddep_launch_dependents();
   if (row >= rows) return;
   constexpr float kLog2e = 1.4426950408889634f;
 

@@ -99,6 +99,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   using L = PrefillSmem<D>;
   constexpr int kHalves = L::kHalves;
   constexpr int kSlots = L::kSlots;
+  // Inputs may come from the kernel before this one in the stream: wait for
+  // it (a no-op unless launched as a programmatic dependent), then let the
+  // next kernel get scheduled as this grid's CTAs finish.
+  griddep_wait();
+  griddep_launch_dependents();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
