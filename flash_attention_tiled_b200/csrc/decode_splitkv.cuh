@@ -43,9 +43,13 @@ constexpr int kDecWarps = 2;          // consumer warps per CTA (a power of two)
 constexpr int kDecPagesPerWarp = 2;   // pages a consumer warp takes per stage
 constexpr int kDecStagePages = kDecWarps * kDecPagesPerWarp;
 constexpr int kDecThreads = 32 * (kDecWarps + 1);
-// Two CTAs share an SM: two independent TMA rings per SM keep more page
-// copies in flight than one ring twice as deep.
+// Up to two CTAs share an SM: two independent TMA rings per SM keep more
+// page copies in flight than one ring twice as deep.  The default grid aims
+// at about 18 MiB of page copies in flight over the whole GPU (192 CTAs of
+// a 96 KB ring); measured on B200, fewer starve HBM of requests and more
+// (two rings on every SM, 28 MiB) read measurably slower.
 constexpr int kDecCtasPerSm = 2;
+constexpr long long kDecInFlightBytes = 18ll << 20;
 constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
 constexpr int kDecMaxBatch = 1024;    // prefix table held in shared memory
 
@@ -587,21 +591,23 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // sum_c 2^(lse_c - M), lse = M + log2 of that denominator, over the CTAs c that
 // held a piece of the segment (M = max lse_c).  Rows are (sequence, query
 // head); CTA x takes rows x, x + grid, ... and first finds, in parallel,
-// which of them belong to split segments.  Inside a row the parts are dealt
-// round-robin to kGroups thread groups (one float4 of the row per thread),
-// each reducing its parts in one pass with a running maximum; the groups'
-// states are then combined through shared memory.
-constexpr int kMergeThreads = 1024;
+// which of them belong to split segments and how many parts the largest has.
+// A thread group (one float4 of a row per thread) reduces its parts in one
+// pass with a running maximum.  Each row gets gpr groups -- enough that a
+// group has at most four parts, so its loads go out together -- and the CTA
+// works on kGroups / gpr rows at once; a row's groups are then combined
+// through shared memory.
+constexpr int kMergeThreads = 512;
 
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kMergeThreads, 2) decode_merge_kernel(const DecodeParams p) {
   constexpr int kV = D / 4;                    // float4 per row
-  constexpr int kGroups = kMergeThreads / kV;  // part groups (32 at D = 128)
+  constexpr int kGroups = kMergeThreads / kV;  // thread groups (16 at D = 128)
   constexpr float kLn2 = 0.69314718055994530942f;
   __shared__ float4 red[kGroups][kV];
   __shared__ float red_m[kGroups], red_s[kGroups];
   __shared__ int list[kMergeThreads];
-  __shared__ int nlist;
+  __shared__ int nlist, max_parts;
   griddep_wait();   // the streaming kernel's partials and segment table
   griddep_launch_dependents();
 
@@ -615,7 +621,10 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
     return b * nseg_b + kvh * p.hgroups + hq / kDecHeadsPerSeg;
   };
   for (long long base = 0; blockIdx.x + base * gridDim.x < rows; base += kMergeThreads) {
-    if (t == 0) nlist = 0;
+    if (t == 0) {
+      nlist = 0;
+      max_parts = 1;
+    }
     __syncthreads();
     const long long row = blockIdx.x + (base + t) * gridDim.x;
     if (row < rows) {
@@ -624,33 +633,61 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
       // (a range outside this grid can only be left over from a call that
       // stopped on a device error; it is skipped so no read leaves the slots)
       const int2 info = p.ws_seg[seg];
-      if (info.x >= 0 && info.x <= info.y && info.y < p.parts) list[atomicAdd(&nlist, 1)] = (int)row;
+      if (info.x >= 0 && info.x <= info.y && info.y < p.parts) {
+        list[atomicAdd(&nlist, 1)] = (int)row;
+        atomicMax(&max_parts, info.y - info.x + 1);
+      }
     }
     __syncthreads();
     const int n = nlist;
-    for (int k = 0; k < n; ++k) {
-      const int row_k = list[k];
-      int r;
-      const int seg = seg_of(row_k, r);
-      const int2 info = p.ws_seg[seg];
-      // this group's parts, one pass with a running maximum (every part
-      // holds at least one key, so its LSE is finite)
+    int gpr = 1;   // groups per row: a power of two with gpr * 4 >= parts
+    while (gpr < kGroups && gpr * 4 < max_parts) gpr <<= 1;
+    const int rpp = kGroups / gpr;               // rows per pass
+    const int slot = grp / gpr, sub = grp % gpr;
+    for (int k0 = 0; k0 < n; k0 += rpp) {
+      const int k = k0 + slot;
       float m = -INFINITY, S = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int cc = info.x + grp; cc <= info.y; cc += kGroups) {
-        const size_t sl = (size_t)(cc + seg) * kDecHeadsPerSeg + r;
-        const float x = p.ws_lse[sl];
-        const float4 v = reinterpret_cast<const float4*>(p.ws_o + sl * D)[l];
-        const float mn = fmaxf(m, x);
-        const float a = fast_exp2(m - mn);   // 0 while m = -inf
-        const float w = fast_exp2(x - mn);
-        S = S * a + w;
-        acc.x = acc.x * a + w * v.x;
-        acc.y = acc.y * a + w * v.y;
-        acc.z = acc.z * a + w * v.z;
-        acc.w = acc.w * a + w * v.w;
-        m = mn;
+      int row_k = -1, seg = 0, r = 0;
+      if (k < n) {
+        row_k = list[k];
+        seg = seg_of(row_k, r);
+        const int2 info = p.ws_seg[seg];
+        // parts sub, sub + gpr, ... in batches of four whose loads are all
+        // issued before any is used; every part holds at least one key, so
+        // its LSE is finite (-inf marks a slot past the last part)
+        for (int c0 = info.x + sub; c0 <= info.y; c0 += 4 * gpr) {
+          float x[4];
+          float4 v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int cc = c0 + j * gpr;
+            x[j] = -INFINITY;
+            v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (cc <= info.y) {
+              const size_t sl = (size_t)(cc + seg) * kDecHeadsPerSeg + r;
+              x[j] = p.ws_lse[sl];
+              v[j] = reinterpret_cast<const float4*>(p.ws_o + sl * D)[l];
+            }
+          }
+          const float mn = fmaxf(fmaxf(m, fmaxf(x[0], x[1])), fmaxf(x[2], x[3]));
+          const float a = fast_exp2(m - mn);   // 0 while m = -inf
+          S *= a;
+          acc.x *= a;
+          acc.y *= a;
+          acc.z *= a;
+          acc.w *= a;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float w = fast_exp2(x[j] - mn);   // 0 for an empty slot
+            S += w;
+            acc.x += w * v[j].x;
+            acc.y += w * v[j].y;
+            acc.z += w * v[j].z;
+            acc.w += w * v[j].w;
+          }
+          m = mn;
+        }
       }
       red[grp][l] = acc;
       if (l == 0) {
@@ -658,17 +695,16 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
         red_s[grp] = S;
       }
       __syncthreads();
-      if (t < kV) {
+      if (sub == 0 && row_k >= 0) {
+        // the row's first group combines the row's gpr groups
         float M = -INFINITY;
-#pragma unroll
-        for (int g2 = 0; g2 < kGroups; ++g2) M = fmaxf(M, red_m[g2]);
+        for (int g2 = grp; g2 < grp + gpr; ++g2) M = fmaxf(M, red_m[g2]);
         float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
         float St = 0.f;
-#pragma unroll 8
-        for (int g2 = 0; g2 < kGroups; ++g2) {
+        for (int g2 = grp; g2 < grp + gpr; ++g2) {
           const float mg = red_m[g2];
           const float w = mg == -INFINITY ? 0.f : fast_exp2(mg - M);   // a group with no part
-          const float4 v = red[g2][t];
+          const float4 v = red[g2][l];
           o4.x += w * v.x;
           o4.y += w * v.y;
           o4.z += w * v.z;
@@ -676,9 +712,9 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
           St += w * red_s[g2];
         }
         const float inv = 1.f / St;
-        *reinterpret_cast<uint2*>(p.o + (size_t)row_k * D + 4 * t) =
+        *reinterpret_cast<uint2*>(p.o + (size_t)row_k * D + 4 * l) =
             make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
-        if (t == 0 && p.lse != nullptr) p.lse[row_k] = (M + fast_log2(St)) * kLn2;
+        if (l == 0 && p.lse != nullptr) p.lse[row_k] = (M + fast_log2(St)) * kLn2;
       }
       __syncthreads();   // red, red_m, red_s reuse
     }

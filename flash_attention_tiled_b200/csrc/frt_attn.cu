@@ -195,7 +195,10 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       frt_status st = device_info(&di);
       if (st != FRT_OK) return st;
     }
-    parts = kDecCtasPerSm * di->sm_count;
+    const long long ring = (D == 128) ? DecodeSmem<128>::kRingBytes : DecodeSmem<64>::kRingBytes;
+    const long long want = (kDecInFlightBytes + ring - 1) / ring;
+    parts = (int)std::min<long long>(std::max<long long>(want, di->sm_count),
+                                     (long long)kDecCtasPerSm * di->sm_count);
   }
   const DecodeWorkspace wl = decode_ws_layout(parts, segments, D);
   if (query) {
@@ -248,8 +251,8 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
     return FRT_ERR_CUDA;
 
   // The merge of split segments: its CTAs are scheduled while the kernel
-  // above still runs and start when it has finished.  One CTA per row, up to
-  // two per SM.
+  // above still runs and start when it has finished.  One CTA per row (two
+  // fit on an SM), at most two per SM.
   const long long rows = (long long)B * Hq;
   const unsigned merge_grid = (unsigned)std::min<long long>(rows, 2ll * di->sm_count);
   const cudaError_t err =

@@ -111,8 +111,10 @@ FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, voi
  *               negative one is read as 0
  *   o           [B, Hq, D] bf16;  lse [B, Hq] fp32, may be NULL
  *   page_size   16 in this version
- *   num_splits  number of work partitions the cache is cut into (0 = two
- *               per SM, the default); every partition streams an equal
+ *   num_splits  number of work partitions the cache is cut into (0 = the
+ *               default: enough partitions for about 18 MiB of page copies
+ *               in flight, 192 on a 148-SM B200, never fewer than one or
+ *               more than two per SM); every partition streams an equal
  *               share of all sequences' pages, so mixed lengths balance
  *   workspace   device scratch of *workspace_bytes bytes, 16-byte aligned.
  *               Size query: a call with q == NULL only writes the required
@@ -191,8 +193,8 @@ FRT_API frt_status frt_attn_prefill_paged(const void* q, const void* k_pages,
  * (held until the process exits).  It allocates nothing and frees nothing.
  *   - Limit: a problem whose workspace (see frt_attn_decode_paged's size
  *     query) exceeds 16 MiB is rejected with FRT_ERR_WORKSPACE before
- *     anything runs.  At D = 128 with two partitions per SM that is roughly
- *     B * Hkv <= 1700 (fewer when a KV head serves more than 16 query heads).
+ *     anything runs.  At D = 128 with the default partitions that is roughly
+ *     B * Hkv <= 1800 (fewer when a KV head serves more than 16 query heads).
  *   - The first call made with a given device current looks up that
  *     device's buffer address; make that first call before any stream
  *     capture on that device.
