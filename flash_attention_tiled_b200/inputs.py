@@ -116,6 +116,45 @@ def paged(B, Hq, Hkv, D, seq_lens=None, len_range=None, page_size=PAGE_SIZE, see
             "page_size": page_size}
 
 
+# e4m3 code that is NaN (sign 0, exponent 15, mantissa 7)
+E4M3_NAN = 0x7F
+E4M3_MAX = 448.0
+
+
+def paged_fp8(B, Hq, Hkv, D, seq_lens=None, len_range=None, page_size=PAGE_SIZE, seed=0,
+              poison=True) -> dict:
+    """A paged FP8 (e4m3) KV cache: the bf16 cache of `paged` with the same
+    seed, stored per KV head as e4m3 codes of value / scale with a power-of-two
+    scale (the smallest with |value| / scale <= 448 over that head's real
+    tokens).  Returns the fields of `paged` with k_pages / v_pages as uint8
+    codes, plus k_scale / v_scale [Hkv] fp32.  The poison page and the tail
+    slots hold the NaN code."""
+    x = paged(B, Hq, Hkv, D, seq_lens=seq_lens, len_range=len_range, page_size=page_size,
+              seed=seed, poison=False)
+    real = x["k_pages"].shape[0] - 1            # the last physical page is the poison page
+    out = dict(x)
+    for name, sname in (("k_pages", "k_scale"), ("v_pages", "v_scale")):
+        t = x[name].float()
+        amax = t[:real].abs().amax(dim=(0, 2, 3)).clamp_min(1e-30)          # [Hkv]
+        sc = torch.exp2(torch.ceil(torch.log2(amax / E4M3_MAX)))
+        codes = (t / sc.view(1, Hkv, 1, 1)).to(torch.float8_e4m3fn).view(torch.uint8)
+        out[name] = codes.contiguous()
+        out[sname] = sc.to(torch.float32)
+    if poison:
+        pp = x["poison_page"]
+        for name in ("k_pages", "v_pages"):
+            out[name][pp] = E4M3_NAN
+        lens = x["seq_lens"]
+        for b in range(B):
+            n = int(lens[b])
+            tail = n % page_size
+            if n > 0 and tail:
+                last = int(x["block_table"][b, (n + page_size - 1) // page_size - 1])
+                out["k_pages"][last, :, tail:, :] = E4M3_NAN
+                out["v_pages"][last, :, tail:, :] = E4M3_NAN
+    return out
+
+
 def make(workload: Workload | str) -> dict:
     """The seeded inputs of one named workload (CPU tensors)."""
     w = WORKLOADS[workload] if isinstance(workload, str) else workload

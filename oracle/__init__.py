@@ -52,9 +52,13 @@ def _load():
         lib.oracle_merge_lse.argtypes = [P, P, I, I, I, P, P]
         lib.oracle_attn_prefill_paged.argtypes = [P, P, P, P, I, P, P, I, I, P, P, I, I, I, I,
                                                   I, I, D]
+        lib.oracle_attn_decode_paged_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, P, P, I, I, I, I,
+                                                     D, P]
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = D
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows,
                   lib.oracle_attn_decode_paged, lib.oracle_merge_lse,
-                  lib.oracle_attn_prefill_paged):
+                  lib.oracle_attn_prefill_paged, lib.oracle_attn_decode_paged_fp8):
             f.restype = I
         _lib = lib
     return _lib
@@ -151,6 +155,41 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, q_lens, causa
                                            _ptr(sl), _ptr(ql), ps, P, _ptr(o), _ptr(lse), B, Hq,
                                            Hkv, max_q, D, int(bool(causal)), float(scale))
     _check(rc, "attn_prefill_paged")
+    return o, lse
+
+
+def e4m3_to_f64(code: int) -> float:
+    """The oracle's FP8 e4m3 decoder for one code (0..255)."""
+    return float(_load().oracle_e4m3_to_f64(int(code)))
+
+
+def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                          scale: float, heads_mask=None):
+    """q [B,Hq,D] bf16; k/v pages [P,Hkv,ps,D] uint8 e4m3 codes; k_scale/v_scale [Hkv]
+    fp32 (KV head h's value = code * scale[h]); block_table [B,maxp]; seq_lens [B].
+    Returns (o [B,Hq,D], lse [B,Hq]) fp64."""
+    B, Hq, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    maxp = bt.shape[1] if bt.ndim == 2 else 0
+    qa = _bits(q)
+    ka = np.ascontiguousarray(k_pages.detach().cpu().numpy(), dtype=np.uint8)
+    va = np.ascontiguousarray(v_pages.detach().cpu().numpy(), dtype=np.uint8)
+    ks = np.ascontiguousarray(np.asarray(k_scale.detach().cpu() if isinstance(k_scale, torch.Tensor)
+                                         else k_scale, dtype=np.float32))
+    vs = np.ascontiguousarray(np.asarray(v_scale.detach().cpu() if isinstance(v_scale, torch.Tensor)
+                                         else v_scale, dtype=np.float32))
+    o = np.zeros((B, Hq, D), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    mask = None
+    if heads_mask is not None:
+        mask = np.ascontiguousarray(np.asarray(heads_mask, dtype=bool).reshape(B, Hq),
+                                    dtype=np.uint8)
+    rc = _load().oracle_attn_decode_paged_fp8(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ks), _ptr(vs),
+                                              _ptr(bt), maxp, _ptr(sl), ps, P, _ptr(o), _ptr(lse),
+                                              B, Hq, Hkv, D, float(scale),
+                                              None if mask is None else _ptr(mask))
+    _check(rc, "attn_decode_paged_fp8")
     return o, lse
 
 

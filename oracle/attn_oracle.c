@@ -309,6 +309,118 @@ int oracle_attn_prefill_paged(const uint16_t *q, const uint16_t *k_pages,
 }
 
 /*
+ * FP8 e4m3 (the "fn" variant: no infinities) to fp64, from its bit fields:
+ * sign s (bit 7), exponent e (bits 6-3, bias 7), mantissa m (bits 2-0).
+ *   e = 0           : (-1)^s * m/8 * 2^(1-7)       (subnormal, zero)
+ *   e = 15, m = 7   : NaN
+ *   otherwise       : (-1)^s * (1 + m/8) * 2^(e-7)
+ * Exported so that the tests can compare it code by code with torch's
+ * float8_e4m3fn.
+ */
+double oracle_e4m3_to_f64(uint8_t code)
+{
+    const int sgn = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m / 8.0, 1 - 7) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -mag : mag;
+}
+
+/* One decode row over fp64 keys and values: scores scale * q.k_j, explicit
+ * softmax, probability-weighted sum of the values (the definition). */
+static void attend_decode_row(const uint16_t *qh, const double *kh, const double *vh, int len,
+                              int D, double scale, double *orow, double *lse, double *s)
+{
+    for (int d = 0; d < D; ++d) orow[d] = 0.0;
+    if (len == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    double m = -INFINITY;
+    for (int j = 0; j < len; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += widen_bf16(qh[d]) * kh[(size_t)j * D + d];
+        s[j] = scale * dot;
+        if (s[j] > m) m = s[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < len; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+    }
+    for (int j = 0; j < len; ++j) {
+        const double w = s[j] / l;
+        for (int d = 0; d < D; ++d) orow[d] += w * vh[(size_t)j * D + d];
+    }
+    *lse = m + log(l);
+}
+
+/*
+ * Paged decode over an FP8 KV cache.  The FasterTransformer read-through
+ * (pptc.cn), section 3.3, stores the KV cache quantised (int8) and
+ * dequantises it before use; section 4.2 enables FP8 on H100 and later.
+ * Reading: K and V pages hold e4m3 codes in the layout of
+ * oracle_attn_decode_paged ([num_pages][Hkv][page_size][D], one byte per
+ * element) and KV head h's value is code * k_scale[h] (resp. v_scale[h]).
+ * The cache is gathered through the block table and dequantised exactly to
+ * fp64, then the same definition applies (Sq = 1, no mask).
+ */
+int oracle_attn_decode_paged_fp8(const uint16_t *q, const uint8_t *k_pages, const uint8_t *v_pages,
+                                 const float *k_scale, const float *v_scale,
+                                 const int32_t *block_table, int max_pages,
+                                 const int32_t *seq_lens, int page_size, int num_pages,
+                                 double *o, double *lse, int B, int Hq, int Hkv, int D,
+                                 double scale, const uint8_t *heads_mask)
+{
+    int rc = check_shape(B, Hq, Hkv, 1, 0, D, scale);
+    if (rc) return rc;
+    if (page_size <= 0 || num_pages < 0 || max_pages < 0) return ORACLE_ERR_ARG;
+    for (int h = 0; h < Hkv; ++h)
+        if (!isfinite(k_scale[h]) || !isfinite(v_scale[h])) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        long long len = seq_lens[b];
+        if (len < 0 || (len + page_size - 1) / page_size > max_pages) return ORACLE_ERR_ARG;
+        for (long long p = 0; p < (len + page_size - 1) / page_size; ++p) {
+            int32_t phys = block_table[(size_t)b * max_pages + p];
+            if (phys < 0 || phys >= num_pages) return ORACLE_ERR_ARG;
+        }
+    }
+    const int g = Hq / Hkv;
+    for (int b = 0; b < B; ++b) {
+        const int len = seq_lens[b];
+        const size_t per_head = (size_t)len * D;
+        double *kc = (double *)malloc(sizeof(double) * (per_head * Hkv + 1));
+        double *vc = (double *)malloc(sizeof(double) * (per_head * Hkv + 1));
+        if (!kc || !vc) { free(kc); free(vc); return ORACLE_ERR_MEM; }
+        for (int kvh = 0; kvh < Hkv; ++kvh)
+            for (int t = 0; t < len; ++t) {
+                const int32_t phys = block_table[(size_t)b * max_pages + t / page_size];
+                const size_t src = (((size_t)phys * Hkv + kvh) * page_size + t % page_size) * D;
+                const size_t dst = (size_t)kvh * per_head + (size_t)t * D;
+                for (int d = 0; d < D; ++d) {
+                    kc[dst + d] = oracle_e4m3_to_f64(k_pages[src + d]) * (double)k_scale[kvh];
+                    vc[dst + d] = oracle_e4m3_to_f64(v_pages[src + d]) * (double)v_scale[kvh];
+                }
+            }
+        int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+        for (int h = 0; h < Hq; ++h) {
+            if (heads_mask && !heads_mask[(size_t)b * Hq + h]) continue;
+            const int kvh = h / g;
+            double *s = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+            if (!s) { failed |= 1; continue; }
+            attend_decode_row(q + ((size_t)b * Hq + h) * D, kc + (size_t)kvh * per_head,
+                              vc + (size_t)kvh * per_head, len, D, scale,
+                              o + ((size_t)b * Hq + h) * D, lse + (size_t)b * Hq + h, s);
+            free(s);
+        }
+        free(kc);
+        free(vc);
+        if (failed) return ORACLE_ERR_MEM;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Merge of partial attention results over disjoint key sets by their
  * log-sum-exp.  If part s attended keys K_s with lse_s = log sum_{j in K_s}
  * exp(s_j) and o_s = sum_{j in K_s} exp(s_j - lse_s) v_j, then over the union

@@ -109,3 +109,44 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, q_lens, causa
                     o[b][h][i][d] = math.fsum(w * r[d] for w, r in zip(weights, rows)) / den
                 lse[b][h][i] = math.log(den)
     return o, lse
+
+
+def e4m3(code: int) -> float:
+    """FP8 e4m3 ("fn": no infinities) code -> float, as an integer significand
+    times a power of two: subnormals m * 2^-9, normals (8 + m) * 2^(e - 10),
+    NaN for exponent 15 with mantissa 7."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 0xF, code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return sign * math.ldexp(m, -9)
+    return sign * math.ldexp(8 + m, e - 10)
+
+
+def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens,
+                          scale: float):
+    """As attn_decode_paged with e4m3 codes in the pages: the value of a cached
+    element of KV head h is e4m3(code) * scale[h], decoded where it is used."""
+    B, Hq, D = len(q), len(q[0]), len(q[0][0])
+    Hkv, ps = len(k_pages[0]), len(k_pages[0][0])
+    group = Hq // Hkv
+    o = [[[0.0] * D for _ in range(Hq)] for _ in range(B)]
+    lse = [[-math.inf] * Hq for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // group
+            weights, rows = [], []
+            for t in range(seq_lens[b]):
+                page = block_table[b][t // ps]
+                key = [e4m3(c) * k_scale[kvh] for c in k_pages[page][kvh][t % ps]]
+                s = scale * math.fsum(q[b][h][d] * key[d] for d in range(D))
+                weights.append(math.exp(s))
+                rows.append([e4m3(c) * v_scale[kvh] for c in v_pages[page][kvh][t % ps]])
+            if not rows:
+                continue
+            den = math.fsum(weights)
+            for d in range(D):
+                o[b][h][d] = math.fsum(w * r[d] for w, r in zip(weights, rows)) / den
+            lse[b][h] = math.log(den)
+    return o, lse

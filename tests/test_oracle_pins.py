@@ -355,3 +355,84 @@ def test_paged_prefill_of_one_token_is_decode():
                                       x["block_table"], x["seq_lens"], 0.25)
     np.testing.assert_array_equal(o[:, :, 0], od)
     np.testing.assert_array_equal(lse[:, :, 0], ld)
+
+
+# ------------------------------------------------------------- FP8 KV cache
+def _torch_e4m3(code: int) -> float:
+    return torch.tensor([code], dtype=torch.uint8).view(torch.float8_e4m3fn).float().item()
+
+
+def test_e4m3_decoder_matches_torch_for_every_code():
+    for c in range(256):
+        got, ref, br = oracle.e4m3_to_f64(c), _torch_e4m3(c), brute.e4m3(c)
+        if math.isnan(ref):
+            assert math.isnan(got) and math.isnan(br), c
+        else:
+            assert got == ref == br, (c, got, ref, br)
+            assert math.copysign(1.0, got) == math.copysign(1.0, ref), c
+
+
+@pytest.mark.parametrize("code,value", [(0x38, 1.0), (0x40, 2.0), (0x7E, 448.0), (0xFE, -448.0),
+                                        (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
+                                        (0x08, 2.0 ** -6), (0x3C, 1.5), (0xB8, -1.0)])
+def test_e4m3_closed_forms(code, value):
+    # e4m3: bias 7, 3 mantissa bits; 0x08 is the smallest normal, 0x7E the largest
+    assert oracle.e4m3_to_f64(code) == value
+
+
+def test_e4m3_nan_and_signed_zero():
+    assert math.isnan(oracle.e4m3_to_f64(0x7F)) and math.isnan(oracle.e4m3_to_f64(0xFF))
+    z = oracle.e4m3_to_f64(0x80)
+    assert z == 0.0 and math.copysign(1.0, z) == -1.0
+
+
+def _fp8_lists(x):
+    return (x["q"].double().tolist(), x["k_pages"].tolist(), x["v_pages"].tolist(),
+            x["block_table"].tolist(), x["seq_lens"].tolist())
+
+
+def test_fp8_paged_decode_matches_brute_force():
+    x = inputs.paged_fp8(2, 4, 2, 8, seq_lens=[7, 9], page_size=4, seed=11)
+    # any scales, not only powers of two; the scales are fp32, so the brute
+    # force gets the same fp32 values
+    ks = torch.tensor([0.37, 1.9], dtype=torch.float32)
+    vs = torch.tensor([0.61, 0.23], dtype=torch.float32)
+    o, l = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"], ks, vs,
+                                        x["block_table"], x["seq_lens"], 0.35)
+    ks, vs = ks.double().tolist(), vs.double().tolist()
+    q, kp, vp, bt, sl = _fp8_lists(x)
+    ob, lb = brute.attn_decode_paged_fp8(q, kp, vp, ks, vs, bt, sl, 0.35)
+    assert np.allclose(o, np.array(ob), rtol=0, atol=1e-12)
+    assert np.allclose(l, np.array(lb), rtol=0, atol=1e-12)
+    assert np.isfinite(o).all()                  # NaN codes in the tails are never read
+
+
+def test_fp8_paged_decode_equals_bf16_decode_on_the_dequantised_cache():
+    # with power-of-two scales every dequantised value is exact in bf16, so the
+    # FP8 path must reproduce the (separately pinned) bf16 oracle
+    x = inputs.paged_fp8(3, 8, 2, 32, seq_lens=[40, 1, 23], page_size=16, seed=12)
+    deq = {}
+    for name, sname in (("k_pages", "k_scale"), ("v_pages", "v_scale")):
+        vals = x[name].view(torch.float8_e4m3fn).double() * x[sname].double().view(1, -1, 1, 1)
+        deq[name] = vals.to(torch.bfloat16)
+        # exact (the NaN codes of the poison page and tail slots stay NaN)
+        assert torch.allclose(deq[name].double(), vals, rtol=0, atol=0, equal_nan=True)
+    o8, l8 = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"], x["k_scale"],
+                                          x["v_scale"], x["block_table"], x["seq_lens"], 0.2)
+    ob, lb = oracle.attn_decode_paged(x["q"], deq["k_pages"], deq["v_pages"], x["block_table"],
+                                      x["seq_lens"], 0.2)
+    assert np.allclose(o8, ob, rtol=0, atol=1e-12)
+    assert np.allclose(l8, lb, rtol=0, atol=1e-12)
+
+
+def test_fp8_scale_enters_linearly():
+    # doubling k_scale doubles every score; doubling v_scale doubles o and
+    # leaves the LSE alone
+    x = inputs.paged_fp8(1, 2, 1, 16, seq_lens=[19], page_size=16, seed=13)
+    args = (x["block_table"], x["seq_lens"])
+    ks, vs = x["k_scale"], x["v_scale"]
+    o1, l1 = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"], ks, vs, *args, 0.5)
+    o2, l2 = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"], ks * 2, vs, *args, 0.25)
+    o3, l3 = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"], ks, vs * 2, *args, 0.5)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    assert np.allclose(2 * o1, o3, atol=1e-12) and np.allclose(l1, l3, atol=1e-12)
