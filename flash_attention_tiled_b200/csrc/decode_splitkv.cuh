@@ -64,19 +64,25 @@ struct DecodeParams {
   int B, Hq, Hkv, g, hgroups;    // g = Hq / Hkv, hgroups = ceil(g / 16)
   int parts;                     // CTAs of the streaming kernel's grid
   float scale_log2;              // scale * log2(e)
+  const float* k_scale;          // FP8 cache: [Hkv] value = code * k_scale[h]; else nullptr
+  const float* v_scale;          // FP8 cache: [Hkv]; else nullptr
   float* ws_o;                   // [slots, 16, D] fp32 partial outputs (normalised)
   float* ws_lse;                 // [slots, 16] fp32 partial LSE (log2 domain)
   int2* ws_seg;                  // [segments] CTAs holding its pieces {first, last};
                                  // {-1, -1}: written out whole (or empty)
 };
 
-template <int D>
+// kFp8: the cache holds FP8 e4m3 codes (one byte per element, D = 128 only):
+// a page is one 16 x 128-byte box; otherwise bf16 pages of D/64 boxes of
+// 16 rows x 64 elements.
+template <int D, bool kFp8 = false>
 struct DecodeSmem {
+  static_assert(!kFp8 || D == 128, "the FP8 cache is supported at D = 128");
   static constexpr int kHalves = D / 64;
-  static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 64 bf16
-  static constexpr int kPageBytes = kHalves * kBoxBytes;              // K or V of one page
+  static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 128 bytes
+  static constexpr int kPageBytes = kDecPage * D * (kFp8 ? 1 : 2);   // K or V of one page
   static constexpr int kStageBytes = kDecStagePages * 2 * kPageBytes; // K+V of 4 pages
-  static constexpr int kStages = (D == 128) ? 3 : 6;                  // 96 KB ring
+  static constexpr int kStages = (96 * 1024) / kStageBytes;           // 96 KB ring
   static constexpr int kRingBytes = kStages * kStageBytes;
   // cross-warp combine: one warp's register state in fragment order
   // (D/16 m-tiles x 2 head tiles x 4 accumulators, then m, l, l_exact for
@@ -123,13 +129,25 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t box_base, int row, int c
   return box_base + row * 128 + ((((col >> 3) ^ (row & 7))) << 4);
 }
 
+// Byte address in a 16 x 128-byte page box written with 128-byte swizzling
+// of the 16-byte chunk `chunk` of row `row`.
+__device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int chunk) {
+  return box_base + row * 128 + (((chunk ^ (row & 7))) << 4);
+}
+
 // kHT: 8-head tiles per segment (1 when a KV head serves at most 8 query
 // heads, else 2; a segment holds at most 16 query heads).
-template <int D, int kHT>
+// kFp8: K/V pages hold e4m3 codes with per-KV-head scales.  The codes become
+// f16 in registers (exact) and the MMAs run in f16; K's scale is folded into
+// the score scale and V's into the final normalisation.  A page's K rows are
+// loaded by ldmatrix as byte quadruples, so the MMA's k index walks d in the
+// order (4c, 4c+1 | 4c+2, 4c+3) per 16-d step, and Q's fragments follow the
+// same order; V^T's rows come out as the even and odd d of each pair.
+template <int D, int kHT, bool kFp8>
 __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using L = DecodeSmem<D>;
+  using L = DecodeSmem<D, kFp8>;
   constexpr int kStages = L::kStages;
   constexpr int kKSteps = D / 16;     // MMA K-steps of K.Q^T
 
@@ -277,8 +295,13 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (lane < n) {
           uint8_t* kdst = ring + stage * L::kStageBytes + lane * 2 * L::kPageBytes;
           uint8_t* vdst = kdst + L::kPageBytes;
-          tma_load_3d(kdst, &tmap_k, &full_bar[stage], 0, row, 0);
-          tma_load_3d(vdst, &tmap_v, &full_bar[stage], 0, row, 0);
+          if constexpr (kFp8) {
+            tma_load_2d(kdst, &tmap_k, &full_bar[stage], 0, row);
+            tma_load_2d(vdst, &tmap_v, &full_bar[stage], 0, row);
+          } else {
+            tma_load_3d(kdst, &tmap_k, &full_bar[stage], 0, row, 0);
+            tma_load_3d(vdst, &tmap_v, &full_bar[stage], 0, row, 0);
+          }
         }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
@@ -313,6 +336,9 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int h0 = kvh * p.g + hg * kDecHeadsPerSeg;            // first query head
     const int nh = min(kDecHeadsPerSeg, p.g - hg * kDecHeadsPerSeg);
     const int len = dec_len_of(p, pc.b);
+    // score scale (exp2 domain) and output scale of this KV head
+    const float sl2 = kFp8 ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
+    const float o_scale = kFp8 ? p.v_scale[kvh] : 1.f;
 
     // Q^T fragments (B operand of S^T = K.Q^T): head 8*ht + r8, d pairs
     uint32_t qb[kHT][kKSteps][2];
@@ -323,8 +349,16 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int head = ht * 8 + r8;
 #pragma unroll
         for (int ks = 0; ks < kKSteps; ++ks) {
-          qb[ht][ks][0] = head < nh ? q32[(head * D + ks * 16 + 2 * qc) / 2] : 0u;
-          qb[ht][ks][1] = head < nh ? q32[(head * D + ks * 16 + 8 + 2 * qc) / 2] : 0u;
+          if constexpr (kFp8) {
+            // d 16ks + 4qc .. +3 as two f16 pairs (the order of the K loads)
+            uint2 w = make_uint2(0u, 0u);
+            if (head < nh) w = *reinterpret_cast<const uint2*>(q32 + (head * D + ks * 16 + 4 * qc) / 2);
+            qb[ht][ks][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+            qb[ht][ks][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+          } else {
+            qb[ht][ks][0] = head < nh ? q32[(head * D + ks * 16 + 2 * qc) / 2] : 0u;
+            qb[ht][ks][1] = head < nh ? q32[(head * D + ks * 16 + 8 + 2 * qc) / 2] : 0u;
+          }
         }
       }
     }
@@ -364,18 +398,40 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           for (int pg = 0; pg < 2; ++pg) {
             if (pg < npg) {
               const uint32_t kbase = base + pg * 2 * L::kPageBytes;
-              uint32_t kf[kKSteps][4];
+              if constexpr (kFp8) {
+                // matrix mi: tokens (mi&1)*8.., 16-byte chunk 2b + (mi>>1); each
+                // ldmatrix covers two K-steps (32 d)
+                uint32_t kr[kKSteps / 2][4];
 #pragma unroll
-              for (int ks = 0; ks < kKSteps; ++ks) {
-                const int col = ks * 16 + (mi >> 1) * 8;
-                ldsm_x4(sw128_addr(kbase + (col >> 6) * L::kBoxBytes, tok, col & 63), kf[ks][0],
-                        kf[ks][1], kf[ks][2], kf[ks][3]);
+                for (int b2 = 0; b2 < kKSteps / 2; ++b2)
+                  ldsm_x4(sw128_chunk(kbase, tok, 2 * b2 + (mi >> 1)), kr[b2][0], kr[b2][1],
+                          kr[b2][2], kr[b2][3]);
+#pragma unroll
+                for (int ks = 0; ks < kKSteps; ++ks) {
+                  const uint32_t r_lo = kr[ks >> 1][(ks & 1) * 2], r_hi = kr[ks >> 1][(ks & 1) * 2 + 1];
+                  uint32_t kf[4];
+                  kf[0] = e4m3x2_to_f16x2(r_lo);         // token r8,   d 4qc, 4qc+1
+                  kf[1] = e4m3x2_to_f16x2(r_hi);         // token r8+8
+                  kf[2] = e4m3x2_to_f16x2(r_lo >> 16);   // token r8,   d 4qc+2, 4qc+3
+                  kf[3] = e4m3x2_to_f16x2(r_hi >> 16);   // token r8+8
+#pragma unroll
+                  for (int ht = 0; ht < kHT; ++ht)
+                    mma_f16_16816(sacc[pg][ht], kf, qb[ht][ks][0], qb[ht][ks][1]);
+                }
+              } else {
+                uint32_t kf[kKSteps][4];
+#pragma unroll
+                for (int ks = 0; ks < kKSteps; ++ks) {
+                  const int col = ks * 16 + (mi >> 1) * 8;
+                  ldsm_x4(sw128_addr(kbase + (col >> 6) * L::kBoxBytes, tok, col & 63), kf[ks][0],
+                          kf[ks][1], kf[ks][2], kf[ks][3]);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kKSteps; ++ks)
+#pragma unroll
+                  for (int ht = 0; ht < kHT; ++ht)
+                    mma_bf16_16816(sacc[pg][ht], kf[ks], qb[ht][ks][0], qb[ht][ks][1]);
               }
-#pragma unroll
-              for (int ks = 0; ks < kKSteps; ++ks)
-#pragma unroll
-                for (int ht = 0; ht < kHT; ++ht)
-                  mma_bf16_16816(sacc[pg][ht], kf[ks], qb[ht][ks][0], qb[ht][ks][1]);
             }
           }
         }
@@ -392,7 +448,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int tok = r8 + (i >> 1) * 8;
-              sc[pg][i] = tok < valid[pg] ? sacc[pg][ht][i] * p.scale_log2 : -INFINITY;
+              sc[pg][i] = tok < valid[pg] ? sacc[pg][ht][i] * sl2 : -INFINITY;
             }
           float e[2][4];
 #pragma unroll
@@ -417,13 +473,24 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
 #pragma unroll
           for (int pg = 0; pg < 2; ++pg) {
-            // rows r8 (lo) and r8+8 (hi) of S^T as bf16 pairs (heads 2qc, 2qc+1)
-            const uint32_t lo = pack_bf16x2(e[pg][0], e[pg][1]);
-            const uint32_t hi = pack_bf16x2(e[pg][2], e[pg][3]);
-            // O is normalised by the bf16-rounded weights that feed P.V; the
-            // LSE uses the exact ones
-            l_run[ht][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
-            l_run[ht][1] += __uint_as_float(lo & 0xffff0000u) + __uint_as_float(hi & 0xffff0000u);
+            // rows r8 (lo) and r8+8 (hi) of S^T as 16-bit pairs (heads 2qc,
+            // 2qc+1): bf16, or f16 for the FP8 cache.  O is normalised by the
+            // rounded weights that feed P.V; the LSE uses the exact ones
+            uint32_t lo, hi;
+            if constexpr (kFp8) {
+              lo = pack_f16x2(e[pg][0], e[pg][1]);
+              hi = pack_f16x2(e[pg][2], e[pg][3]);
+              float a0, a1, b0, b1;
+              unpack_f16x2(lo, a0, a1);
+              unpack_f16x2(hi, b0, b1);
+              l_run[ht][0] += a0 + b0;
+              l_run[ht][1] += a1 + b1;
+            } else {
+              lo = pack_bf16x2(e[pg][0], e[pg][1]);
+              hi = pack_bf16x2(e[pg][2], e[pg][3]);
+              l_run[ht][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
+              l_run[ht][1] += __uint_as_float(lo & 0xffff0000u) + __uint_as_float(hi & 0xffff0000u);
+            }
             le_run[ht][0] += e[pg][0] + e[pg][2];
             le_run[ht][1] += e[pg][1] + e[pg][3];
             // transpose to the B layout of P^T (token pairs, head r8)
@@ -446,7 +513,48 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         // ---- O^T += V^T.P^T per page: V^T fragments by transposing ldmatrix
-        {
+        if constexpr (kFp8) {
+          // matrix mi: tokens (mi&1)*8.., 16-byte chunk 2u + (mi>>1).  A
+          // transposed word holds tokens 2qc, 2qc+1 of d pair (2r8, 2r8+1);
+          // the byte permute splits it into the even-d pair (row r8 of the
+          // m-tile) and the odd-d pair (row r8+8)
+          const int mi = lane >> 3, j = lane & 7;
+          const int tok = (mi & 1) * 8 + j;
+#pragma unroll
+          for (int pg = 0; pg < 2; ++pg) {
+            if (pg < npg) {
+              const uint32_t vbase = base + pg * 2 * L::kPageBytes + L::kPageBytes;
+              uint32_t vr[kMT / 2][4];
+#pragma unroll
+              for (int u = 0; u < kMT / 2; ++u)
+                ldsm_x4_trans(sw128_chunk(vbase, tok, 2 * u + (mi >> 1)), vr[u][0], vr[u][1],
+                              vr[u][2], vr[u][3]);
+              const int v = valid[pg];
+              const int t0 = 2 * qc;
+              const uint32_t m01 = (t0 < v ? 0xffffu : 0u) | (t0 + 1 < v ? 0xffff0000u : 0u);
+              const uint32_t m89 = (t0 + 8 < v ? 0xffffu : 0u) | (t0 + 9 < v ? 0xffff0000u : 0u);
+#pragma unroll
+              for (int mt = 0; mt < kMT; ++mt) {
+                const uint32_t w0 = prmt_b32(vr[mt >> 1][(mt & 1) * 2], 0x3120u);       // tokens 2qc..
+                const uint32_t w8 = prmt_b32(vr[mt >> 1][(mt & 1) * 2 + 1], 0x3120u);   // tokens 8+2qc..
+                uint32_t vf[4];
+                vf[0] = e4m3x2_to_f16x2(w0);          // d 16mt + 2r8,     tokens 2qc, 2qc+1
+                vf[1] = e4m3x2_to_f16x2(w0 >> 16);    // d 16mt + 2r8 + 1
+                vf[2] = e4m3x2_to_f16x2(w8);          // d 16mt + 2r8,     tokens 8+2qc, 9+2qc
+                vf[3] = e4m3x2_to_f16x2(w8 >> 16);    // d 16mt + 2r8 + 1
+                if (v < kDecPage) {   // tokens past the sequence end may hold anything (NaN)
+                  vf[0] &= m01;
+                  vf[1] &= m01;
+                  vf[2] &= m89;
+                  vf[3] &= m89;
+                }
+#pragma unroll
+                for (int ht = 0; ht < kHT; ++ht)
+                  mma_f16_16816(acc[mt][ht], vf, pbf[pg][ht][0], pbf[pg][ht][1]);
+              }
+            }
+          }
+        } else         {
           const int mi = lane >> 3, j = lane & 7;
           const int tok = (mi >> 1) * 8 + j;
 #pragma unroll
@@ -558,22 +666,34 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           const int r = ht * 8 + 2 * qc + hh;   // head within the segment
           if (r < nh) {
-            const float inv = 1.f / ls;
+            const float inv = o_scale / ls;
             const float lse2 = m_run[ht][hh] + fast_log2(le);
+            // m-tile row r8 / r8+8 is d 16mt + r8 / + 8 (bf16 cache), or the
+            // pair d 16mt + 2r8, + 1 (FP8 cache)
             if (whole) {
               __nv_bfloat16* orow = p.o + ((size_t)pc.b * p.Hq + h0 + r) * D;
 #pragma unroll
               for (int mt = 0; mt < kMT; ++mt) {
-                orow[mt * 16 + r8] = __float2bfloat16(acc[mt][ht][hh] * inv);
-                orow[mt * 16 + 8 + r8] = __float2bfloat16(acc[mt][ht][2 + hh] * inv);
+                if constexpr (kFp8) {
+                  *reinterpret_cast<uint32_t*>(orow + mt * 16 + 2 * r8) =
+                      pack_bf16x2(acc[mt][ht][hh] * inv, acc[mt][ht][2 + hh] * inv);
+                } else {
+                  orow[mt * 16 + r8] = __float2bfloat16(acc[mt][ht][hh] * inv);
+                  orow[mt * 16 + 8 + r8] = __float2bfloat16(acc[mt][ht][2 + hh] * inv);
+                }
               }
               if (r8 == 0 && p.lse != nullptr) p.lse[(size_t)pc.b * p.Hq + h0 + r] = lse2 * kLn2;
             } else {
               float* orow = p.ws_o + ((size_t)slot * kDecHeadsPerSeg + r) * D;
 #pragma unroll
               for (int mt = 0; mt < kMT; ++mt) {
-                orow[mt * 16 + r8] = acc[mt][ht][hh] * inv;
-                orow[mt * 16 + 8 + r8] = acc[mt][ht][2 + hh] * inv;
+                if constexpr (kFp8) {
+                  *reinterpret_cast<float2*>(orow + mt * 16 + 2 * r8) =
+                      make_float2(acc[mt][ht][hh] * inv, acc[mt][ht][2 + hh] * inv);
+                } else {
+                  orow[mt * 16 + r8] = acc[mt][ht][hh] * inv;
+                  orow[mt * 16 + 8 + r8] = acc[mt][ht][2 + hh] * inv;
+                }
               }
               if (r8 == 0) p.ws_lse[(size_t)slot * kDecHeadsPerSeg + r] = lse2;
             }

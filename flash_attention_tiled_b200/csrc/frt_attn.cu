@@ -46,18 +46,24 @@ frt_status device_info(DeviceInfo** out) {
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FRT_ERR_CUDA;
       di.sm_count = sms;
-      if (cudaFuncSetAttribute(decode_splitkv_kernel<128, 1>,
+      if (cudaFuncSetAttribute(decode_splitkv_kernel<128, 1, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<128>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(decode_splitkv_kernel<128, 2>,
+          cudaFuncSetAttribute(decode_splitkv_kernel<128, 2, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<128>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(decode_splitkv_kernel<64, 1>,
+          cudaFuncSetAttribute(decode_splitkv_kernel<64, 1, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<64>::kBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(decode_splitkv_kernel<64, 2>,
+          cudaFuncSetAttribute(decode_splitkv_kernel<64, 2, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DecodeSmem<64>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(decode_splitkv_kernel<128, 1, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<128, true>::kBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(decode_splitkv_kernel<128, 2, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeSmem<128, true>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(prefill_kernel<128, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrefillSmem<128>::kBytes) != cudaSuccess ||
@@ -110,10 +116,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 128-byte swizzling.  dims/box are innermost first;
-// strides_bytes[i] is the stride of dims[i + 1].
+// Tensor map (bf16 unless told otherwise) with 128-byte swizzling.  dims/box
+// are innermost first; strides_bytes[i] is the stride of dims[i + 1].
 bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-               const uint64_t* strides_bytes, const uint32_t* box) {
+               const uint64_t* strides_bytes, const uint32_t* box,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t gdim[5], gstr[4];
@@ -124,7 +131,7 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dim
     estr[i] = 1;
     if (i + 1 < rank) gstr[i] = strides_bytes[i];
   }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+  CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void*>(base),
                   gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -179,7 +186,9 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
                          uint64_t cache_rows, const int32_t* block_table, int max_pages,
                          const int32_t* seq_lens, int contig_len, void* o, float* lse, int B,
                          int Hq, int Hkv, int D, float scale, int num_splits, void* workspace,
-                         size_t* workspace_bytes, cudaStream_t stream) {
+                         size_t* workspace_bytes, cudaStream_t stream, bool fp8 = false,
+                         const float* k_scale = nullptr, const float* v_scale = nullptr) {
+  // fp8: the pages hold e4m3 codes with per-KV-head scales (D = 128)
   const bool query = (q == nullptr);
   DeviceInfo* di = nullptr;
   if (!query) {
@@ -195,7 +204,8 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       frt_status st = device_info(&di);
       if (st != FRT_OK) return st;
     }
-    const long long ring = (D == 128) ? DecodeSmem<128>::kRingBytes : DecodeSmem<64>::kRingBytes;
+    const long long ring = fp8 ? DecodeSmem<128, true>::kRingBytes
+                               : (D == 128) ? DecodeSmem<128>::kRingBytes : DecodeSmem<64>::kRingBytes;
     const long long want = (kDecInFlightBytes + ring - 1) / ring;
     parts = (int)std::min<long long>(std::max<long long>(want, di->sm_count),
                                      (long long)kDecCtasPerSm * di->sm_count);
@@ -211,16 +221,26 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       !aligned16(workspace))
     return FRT_ERR_WORKSPACE;
 
-  // One TMA box per page: (64 columns, 16 rows, D/64 column halves).  The
-  // half index is the outermost box dimension, so the page lands in shared
-  // memory as D/64 consecutive 16x64 swizzled blocks.
+  // One TMA box per page.  bf16: (64 columns, 16 rows, D/64 column halves);
+  // the half index is the outermost box dimension, so the page lands in
+  // shared memory as D/64 consecutive 16x64 swizzled blocks.  FP8: one box of
+  // 16 rows x 128 bytes.
   CUtensorMap tk, tv;
-  const uint64_t dims[3] = {64, cache_rows, (uint64_t)(D / 64)};
-  const uint64_t strides[2] = {(uint64_t)D * 2, 128};
-  const uint32_t box[3] = {64, (uint32_t)kDecPage, (uint32_t)(D / 64)};
-  if (!make_tmap(&tk, k_base, 3, dims, strides, box) ||
-      !make_tmap(&tv, v_base, 3, dims, strides, box))
-    return FRT_ERR_CUDA;
+  if (fp8) {
+    const uint64_t dims[2] = {(uint64_t)D, cache_rows};
+    const uint64_t strides[1] = {(uint64_t)D};
+    const uint32_t box[2] = {(uint32_t)D, (uint32_t)kDecPage};
+    if (!make_tmap(&tk, k_base, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8) ||
+        !make_tmap(&tv, v_base, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return FRT_ERR_CUDA;
+  } else {
+    const uint64_t dims[3] = {64, cache_rows, (uint64_t)(D / 64)};
+    const uint64_t strides[2] = {(uint64_t)D * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)kDecPage, (uint32_t)(D / 64)};
+    if (!make_tmap(&tk, k_base, 3, dims, strides, box) ||
+        !make_tmap(&tv, v_base, 3, dims, strides, box))
+      return FRT_ERR_CUDA;
+  }
 
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -237,6 +257,8 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
   p.hgroups = hgroups;
   p.parts = parts;
   p.scale_log2 = scale * kLog2e;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
@@ -244,9 +266,12 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
 
   // one 8-head tile per segment when a KV head serves at most 8 query heads
   const bool one_tile = g <= 8;
-  const size_t smem = (D == 128) ? DecodeSmem<128>::kBytes : DecodeSmem<64>::kBytes;
-  auto* kernel = (D == 128) ? (one_tile ? decode_splitkv_kernel<128, 1> : decode_splitkv_kernel<128, 2>)
-                            : (one_tile ? decode_splitkv_kernel<64, 1> : decode_splitkv_kernel<64, 2>);
+  const size_t smem = fp8 ? DecodeSmem<128, true>::kBytes
+                          : (D == 128) ? DecodeSmem<128>::kBytes : DecodeSmem<64>::kBytes;
+  auto* kernel =
+      fp8 ? (one_tile ? decode_splitkv_kernel<128, 1, true> : decode_splitkv_kernel<128, 2, true>)
+      : (D == 128) ? (one_tile ? decode_splitkv_kernel<128, 1, false> : decode_splitkv_kernel<128, 2, false>)
+                   : (one_tile ? decode_splitkv_kernel<64, 1, false> : decode_splitkv_kernel<64, 2, false>);
   if (launch_pdl(kernel, dim3(parts), dim3(kDecThreads), smem, stream, tk, tv, p) != cudaSuccess)
     return FRT_ERR_CUDA;
 
@@ -373,6 +398,17 @@ __global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
   }
 }
 
+__global__ void fp8_decode_selftest_kernel(const uint8_t* codes, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i < n) {
+    const uint32_t x = codes[i] | (i + 1 < n ? (uint32_t)codes[i + 1] << 8 : 0u);
+    float lo, hi;
+    unpack_f16x2(e4m3x2_to_f16x2(x), lo, hi);
+    y[i] = lo;
+    if (i + 1 < n) y[i + 1] = hi;
+  }
+}
+
 }  // namespace
 }  // namespace frt
 
@@ -407,6 +443,38 @@ frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void*
   return launch_decode(q, k_pages, v_pages, (uint64_t)num_pages * Hkv * page_size, block_table,
                        max_pages_per_seq, seq_lens, 0, o, lse, B, Hq, Hkv, D, scale,
                        num_splits, workspace, workspace_bytes, stream);
+}
+
+frt_status frt_attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages,
+                                     const float* k_scale, const float* v_scale,
+                                     const int32_t* block_table, int max_pages_per_seq,
+                                     const int32_t* seq_lens, int page_size, int num_pages,
+                                     void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                     float scale, int num_splits, void* workspace,
+                                     size_t* workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq < 0 ||
+      num_splits < 0 || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 128) return FRT_ERR_UNSUPPORTED;
+  if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
+  if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  if (q != nullptr && B > 0) {
+    if (k_pages == nullptr || v_pages == nullptr || o == nullptr || k_scale == nullptr ||
+        v_scale == nullptr || seq_lens == nullptr ||
+        (block_table == nullptr && max_pages_per_seq > 0))
+      return FRT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
+        (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+      return FRT_ERR_INVALID_ARG;
+    if (num_pages == 0) return FRT_ERR_INVALID_ARG;
+  }
+  return launch_decode(q, k_pages, v_pages, (uint64_t)num_pages * Hkv * page_size, block_table,
+                       max_pages_per_seq, seq_lens, 0, o, lse, B, Hq, Hkv, D, scale, num_splits,
+                       workspace, workspace_bytes, stream, true, k_scale, v_scale);
 }
 
 frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -525,6 +593,14 @@ frt_status frt_read_device_error(unsigned* flags) {
     return FRT_ERR_CUDA;
   *flags = v;
   return FRT_OK;
+}
+
+frt_status frt_debug_fp8_decode(const uint8_t* codes, float* y, int n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (codes == nullptr || y == nullptr))) return FRT_ERR_INVALID_ARG;
+  if (n == 0) return FRT_OK;
+  const int pairs = (n + 1) / 2;
+  fp8_decode_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(codes, y, n);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 
 frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {

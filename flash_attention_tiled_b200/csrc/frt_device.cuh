@@ -230,6 +230,46 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// D(16x8, fp32) += A(16x16, f16, row) * B(16x8, f16, col)
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0,
+                                              uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// the two halves of an f16x2 as floats (exact)
+__device__ __forceinline__ void unpack_f16x2(uint32_t x, float& lo, float& hi) {
+  uint16_t l, h;
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(l), "=h"(h) : "r"(x));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(l));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(h));
+}
+
+// Two FP8 e4m3 codes (bits 0-7 and 8-15 of x) -> f16x2 with the code in bits
+// 0-7 in the low half.  Every e4m3 value is exact in f16.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
+  uint32_t d;
+  const uint16_t h = (uint16_t)(x & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(h));
+  return d;
+}
+
+// byte permute of one word: result byte i = byte (sel >> 4i) & 7 of {x, 0}
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t x, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(x), "r"(sel));
+  return d;
+}
+
 // max of three (sm_100 three-input form)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;

@@ -17,9 +17,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
 EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
-           "frt_attn_prefill_paged",
+           "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8",
            "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
-           "frt_version")
+           "frt_debug_fp8_decode", "frt_version")
 
 STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
           3: "FRT_ERR_WORKSPACE", 4: "FRT_ERR_CUDA"}
@@ -47,6 +47,9 @@ def _load() -> ctypes.CDLL:
                                            P]
     lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.frt_debug_exp2_poly.argtypes = [P, P, I, P]
+    lib.frt_attn_decode_paged_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I,
+                                              P, Z, P]
+    lib.frt_debug_fp8_decode.argtypes = [P, P, I, P]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = ctypes.c_int
     lib.frt_version.restype = ctypes.c_char_p
@@ -163,6 +166,53 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
         _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale, num_splits,
         _ptr(ws), ctypes.byref(need), stream))
     return out, lse
+
+
+def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                          k_scale: torch.Tensor, v_scale: torch.Tensor,
+                          block_table: torch.Tensor, seq_lens: torch.Tensor,
+                          scale: float | None = None, num_splits: int = 0,
+                          out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                          return_lse: bool = True):
+    """o, lse = decode attention of q [B,Hq,D] (bf16) over an FP8 cache: pages
+    [P,Hkv,ps,D] of e4m3 codes (uint8), KV head h's values = code * scale[h]
+    with k_scale / v_scale [Hkv] fp32."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.uint8, 4)
+    _need(v_pages, "v_pages", torch.uint8, 4)
+    _need(k_scale, "k_scale", torch.float32, 1)
+    _need(v_scale, "v_scale", torch.float32, 1)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    P, Hkv, ps, _ = k_pages.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    stream = _stream(q.device)
+    need = ctypes.c_size_t(0)
+    _check("frt_attn_decode_paged_fp8", _lib.frt_attn_decode_paged_fp8(
+        None, None, None, None, None, None, block_table.shape[1], None, ps, P, None, None, B, Hq,
+        Hkv, D, scale, num_splits, None, ctypes.byref(need), stream))
+    ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, num_splits, "fp8"))
+    need = ctypes.c_size_t(ws.numel())
+    _check("frt_attn_decode_paged_fp8", _lib.frt_attn_decode_paged_fp8(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale,
+        num_splits, _ptr(ws), ctypes.byref(need), stream))
+    return out, lse
+
+
+def debug_fp8_decode(codes: torch.Tensor) -> torch.Tensor:
+    """The FP8 decode kernel's conversion of e4m3 codes (uint8, on the device)."""
+    _need(codes, "codes", torch.uint8, 1)
+    y = torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    _check("frt_debug_fp8_decode", _lib.frt_debug_fp8_decode(
+        _ptr(codes), _ptr(y), codes.numel(), _stream(codes.device)))
+    return y
 
 
 def attn_decode_paged_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,

@@ -213,6 +213,33 @@ FRT_API frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pa
                                                  cudaStream_t stream);
 
 /*
+ * frt_attn_decode_paged_fp8 -- frt_attn_decode_paged over an FP8 KV cache.
+ * The FasterTransformer read-through (pptc.cn) keeps the KV cache quantised
+ * and dequantises it before use (section 3.3, an int8 KV cache) and enables
+ * FP8 on H100 and later (section 4.2).  Here the pages hold e4m3 codes
+ * (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities;
+ * 0x7F / 0xFF are NaN), one byte per element, in the layout of
+ * frt_attn_decode_paged: [num_pages, Hkv, page_size, D] uint8.  An element
+ * of KV head h stands for code * k_scale[h] (keys) or code * v_scale[h]
+ * (values); every other argument means what it means for
+ * frt_attn_decode_paged, and the workspace size query is the same.
+ *   k_scale, v_scale  [Hkv] fp32 on the device, finite, 4-byte aligned
+ *   D                 128 only (FRT_ERR_UNSUPPORTED otherwise)
+ * The kernel converts codes to f16 (exact), multiplies q.k in f16 with fp32
+ * accumulation, and rounds the softmax weights to f16 before P.V; the scales
+ * are applied in fp32 to the scores and to the output.  Tail slots and pages
+ * past a sequence's length may hold NaN codes: they never reach o.
+ */
+FRT_API frt_status frt_attn_decode_paged_fp8(const void* q, const void* k_pages,
+                                             const void* v_pages, const float* k_scale,
+                                             const float* v_scale, const int32_t* block_table,
+                                             int max_pages_per_seq, const int32_t* seq_lens,
+                                             int page_size, int num_pages, void* o, float* lse,
+                                             int B, int Hq, int Hkv, int D, float scale,
+                                             int num_splits, void* workspace,
+                                             size_t* workspace_bytes, cudaStream_t stream);
+
+/*
  * frt_attn_merge_lse -- combine S partial attention results of the same rows,
  * each computed over a disjoint set of keys, into the result over their
  * union.  This is the correct form of the per-page combination in the
@@ -241,10 +268,19 @@ FRT_API frt_status frt_read_device_error(unsigned* flags);
 /*
  * frt_debug_exp2_poly -- diagnostic: y[i] = the library's FMA-pipe 2^x for
  * x[i] (device arrays of n floats; inputs below -125 are clamped there).
- * The prefill kernel computes a quarter of its softmax exponentials this
- * way; tests compare it with CUDA's exp2f.  Not part of the attention path.
+ * The prefill kernel's softmax can compute part of its exponentials this way
+ * (a compile-time option, off in this build); tests compare it with CUDA's
+ * exp2f.  Not part of the attention path.
  */
 FRT_API frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
+/*
+ * frt_debug_fp8_decode -- diagnostic: y[i] = the value of e4m3 code codes[i]
+ * as the FP8 decode kernel converts it (device arrays of n elements).  Tests
+ * compare it with the e4m3 definition.  Not part of the attention path.
+ */
+FRT_API frt_status frt_debug_fp8_decode(const uint8_t* codes, float* y, int n,
+                                        cudaStream_t stream);
 
 /* Library version string ("major.minor.patch"). */
 FRT_API const char* frt_version(void);

@@ -98,3 +98,40 @@ def test_merge_rejects(S, B, Hq, D, code):
 
 def test_merge_empty_rows_is_a_noop():
     assert frt.lib().frt_attn_merge_lse(NULL, NULL, 3, 0, 4, 64, NULL, NULL, NULL) == 0
+
+
+def _fp8(B=1, Hq=8, Hkv=2, D=128, page_size=16, scale=0.1, num_pages=10, splits=0,
+         q=NULL, ks=NULL, vs=NULL):
+    need = Z(0)
+    fake = ctypes.c_void_p(256)            # aligned, never dereferenced: rejected first
+    args = (q, fake if q else NULL, fake if q else NULL, ks, vs, fake if q else NULL, 4,
+            fake if q else NULL, page_size, num_pages, fake if q else NULL, NULL, B, Hq, Hkv, D,
+            scale, splits, NULL, ctypes.byref(need), NULL)
+    return frt.lib().frt_attn_decode_paged_fp8(*args), need.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), 1),
+    (dict(D=64), 2),                      # the FP8 cache is built for D = 128
+    (dict(page_size=8), 2),
+    (dict(scale=0.0), 1),
+    (dict(B=-1), 1),
+    (dict(q=ctypes.c_void_p(256)), 1),    # a real call without scales
+])
+def test_decode_fp8_rejects(kw, code):
+    rc, _ = _fp8(**kw)
+    assert rc == code
+
+
+def test_decode_fp8_workspace_query_matches_bf16():
+    rc, need8 = _fp8(B=3, Hq=16, Hkv=4, splits=37)
+    assert rc == 0
+    need = Z(0)
+    rc = frt.lib().frt_attn_decode_paged(NULL, NULL, NULL, NULL, 4, NULL, 16, 10, NULL, NULL, 3,
+                                         16, 4, 128, 0.1, 37, NULL, ctypes.byref(need), NULL)
+    assert rc == 0 and need.value == need8
+
+
+def test_debug_fp8_decode_rejects():
+    assert frt.lib().frt_debug_fp8_decode(NULL, NULL, -1, NULL) == 1
+    assert frt.lib().frt_debug_fp8_decode(NULL, NULL, 0, NULL) == 0

@@ -264,6 +264,102 @@ def test_decode_splits_agree(frt):
         assert (l1 - l2).abs().max().item() <= 1e-4
 
 
+# ------------------------------------------------------ FP8 (e4m3) KV cache
+def test_fp8_conversion_matches_the_e4m3_definition(frt):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    y = frt.debug_fp8_decode(codes.cuda()).cpu()
+    for c in range(256):
+        ref = oracle.e4m3_to_f64(c)
+        if math.isnan(ref):
+            assert math.isnan(y[c].item()), c
+        else:
+            assert y[c].item() == ref, (c, y[c].item(), ref)
+
+
+def _fp8_case(frt, x, scale, num_splits=0, what=""):
+    d = _dev(x)
+    o, lse = frt.attn_decode_paged_fp8(d["q"], d["k_pages"], d["v_pages"], d["k_scale"],
+                                       d["v_scale"], d["block_table"], d["seq_lens"],
+                                       scale=scale, num_splits=num_splits)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_decode_paged_fp8(x["q"], x["k_pages"], x["v_pages"],
+                                                  x["k_scale"], x["v_scale"], x["block_table"],
+                                                  x["seq_lens"], scale)
+    _compare(o, o_ref, lse, lse_ref, what)
+    return o, lse
+
+
+@pytest.mark.parametrize("name", ["paged_gqa_decode_b4", "long_splitkv_decode_256k"])
+def test_fp8_paged_decode_workloads(frt, name):
+    # the named paged workloads with their cache stored as e4m3 (per-KV-head
+    # power-of-two scales); NaN codes in the poison page and tail slots
+    w = inputs.WORKLOADS[name]
+    x = inputs.paged_fp8(w.B, w.Hq, w.Hkv, w.D, len_range=w.len_range, page_size=w.page_size,
+                         seed=w.seed)
+    _fp8_case(frt, x, w.scale, what=f"fp8 {name}")
+    _no_device_error(frt)
+
+
+FP8_CASES = [  # lens, Hq, Hkv, num_splits
+    ([1], 8, 8, 0),
+    ([15, 16, 17, 33], 8, 2, 0),
+    ([5000, 0, 300], 32, 4, 0),           # an empty sequence
+    ([4096], 32, 1, 0),                   # MQA, two head groups of 16
+    ([3333, 77], 24, 2, 1),               # one partition: no merge
+    ([3333, 77], 24, 2, 1000),            # more partitions than pages
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=str)
+def test_fp8_decode_edge(frt, case):
+    lens, Hq, Hkv, splits = case
+    x = inputs.paged_fp8(len(lens), Hq, Hkv, 128, seq_lens=lens, seed=len(lens) * 17 + Hq)
+    o, lse = _fp8_case(frt, x, 1.0 / math.sqrt(128), splits, f"fp8 {case}")
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
+    _no_device_error(frt)
+
+
+@pytest.mark.parametrize("t_star", [0, 17, 4095, 4099])
+def test_fp8_decode_page_indexing_probe(frt, t_star):
+    # keys 0 except token t*, whose key code is 448 on d 0: p is one-hot and o
+    # must be that token's dequantised value row exactly
+    B, Hq, Hkv, D, n = 2, 8, 2, 128, 4100
+    x = inputs.paged_fp8(B, Hq, Hkv, D, seq_lens=[n, n - 37], seed=t_star)
+    q = torch.zeros_like(x["q"])
+    q[:, :, 0] = 1.0
+    kp = torch.zeros_like(x["k_pages"])
+    for b in range(B):
+        if t_star < int(x["seq_lens"][b]):
+            kp[int(x["block_table"][b, t_star // 16]), :, t_star % 16, 0] = 0x7E
+    x["q"], x["k_pages"] = q, kp
+    x["k_scale"] = torch.ones(Hkv)
+    d = _dev(x)
+    o, _ = frt.attn_decode_paged_fp8(d["q"], d["k_pages"], d["v_pages"], d["k_scale"],
+                                     d["v_scale"], d["block_table"], d["seq_lens"], scale=1.0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        if t_star >= int(x["seq_lens"][b]):
+            continue
+        phys = int(x["block_table"][b, t_star // 16])
+        for h in range(Hq):
+            kvh = h // (Hq // Hkv)
+            row = x["v_pages"][phys, kvh, t_star % 16].view(torch.float8_e4m3fn).float()
+            ref = (row * x["v_scale"][kvh]).to(torch.bfloat16)
+            assert torch.equal(o[b, h].cpu(), ref)
+
+
+def test_fp8_decode_deterministic(frt):
+    x = _dev(inputs.paged_fp8(3, 16, 2, 128, seq_lens=[9000, 100, 20000], seed=5))
+    args = (x["q"], x["k_pages"], x["v_pages"], x["k_scale"], x["v_scale"], x["block_table"],
+            x["seq_lens"])
+    o1, l1 = frt.attn_decode_paged_fp8(*args)
+    o2, l2 = frt.attn_decode_paged_fp8(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 # ------------------------------------------------------------------- merge
 @pytest.mark.parametrize("S,B,Hq,D,empty", [(1, 2, 8, 128, 0.0), (5, 3, 16, 128, 0.3),
                                             (37, 1, 32, 128, 0.0), (4, 2, 4, 64, 0.5)])
