@@ -39,10 +39,16 @@
 namespace frt {
 
 constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
-constexpr int kDecWarps = 2;          // consumer warps per CTA (a power of two)
 constexpr int kDecPagesPerWarp = 2;   // pages a consumer warp takes per stage
-constexpr int kDecStagePages = kDecWarps * kDecPagesPerWarp;
-constexpr int kDecThreads = 32 * (kDecWarps + 1);
+// Consumer warps per CTA (a power of two): 4 for an FP8 cache with one 8-head
+// tile (a stage of 8 FP8 pages is 32 KB, and the consumers, not HBM, set the
+// pace), else 2.
+template <bool kFp8, int kHT>
+struct DecodeCfg {
+  static constexpr int kWarps = (kFp8 && kHT == 1) ? 4 : 2;
+  static constexpr int kStagePages = kWarps * kDecPagesPerWarp;
+  static constexpr int kThreads = 32 * (kWarps + 1);
+};
 // Up to two CTAs share an SM: two independent TMA rings per SM keep more
 // page copies in flight than one ring twice as deep.  The default grid aims
 // at about 18 MiB of page copies in flight over the whole GPU (192 CTAs of
@@ -75,20 +81,21 @@ struct DecodeParams {
 // kFp8: the cache holds FP8 e4m3 codes (one byte per element, D = 128 only):
 // a page is one 16 x 128-byte box; otherwise bf16 pages of D/64 boxes of
 // 16 rows x 64 elements.
-template <int D, bool kFp8 = false>
+template <int D, bool kFp8 = false, int kHT = 2>
 struct DecodeSmem {
   static_assert(!kFp8 || D == 128, "the FP8 cache is supported at D = 128");
+  using Cfg = DecodeCfg<kFp8, kHT>;
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 128 bytes
   static constexpr int kPageBytes = kDecPage * D * (kFp8 ? 1 : 2);   // K or V of one page
-  static constexpr int kStageBytes = kDecStagePages * 2 * kPageBytes; // K+V of 4 pages
+  static constexpr int kStageBytes = Cfg::kStagePages * 2 * kPageBytes; // K+V of a stage
   static constexpr int kStages = (96 * 1024) / kStageBytes;           // 96 KB ring
   static constexpr int kRingBytes = kStages * kStageBytes;
   // cross-warp combine: one warp's register state in fragment order
-  // (D/16 m-tiles x 2 head tiles x 4 accumulators, then m, l, l_exact for
-  // 2 heads of each head tile), sized for two head tiles
-  static constexpr int kFragFloats = (D / 16) * 2 * 4 + 12;
-  static constexpr int kScratchFloats = (kDecWarps / 2) * kFragFloats * 32;
+  // (D/16 m-tiles x kHT head tiles x 4 accumulators, then m, l, l_exact for
+  // 2 heads of each head tile)
+  static constexpr int kFragFloats = (D / 16) * kHT * 4 + 6 * kHT;
+  static constexpr int kScratchFloats = (Cfg::kWarps / 2) * kFragFloats * 32;
   static constexpr int kScratchOff = kRingBytes;
   static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
   static constexpr int kBarOff = kPrefixOff + ((kDecMaxBatch + 1) * 4 + 15) / 16 * 16;
@@ -144,10 +151,12 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int 
 // order (4c, 4c+1 | 4c+2, 4c+3) per 16-d step, and Q's fragments follow the
 // same order; V^T's rows come out as the even and odd d of each pair.
 template <int D, int kHT, bool kFp8>
-__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
+__global__ void __launch_bounds__(DecodeCfg<kFp8, kHT>::kThreads, kDecCtasPerSm)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using L = DecodeSmem<D, kFp8>;
+  using L = DecodeSmem<D, kFp8, kHT>;
+  constexpr int kDecWarps = DecodeCfg<kFp8, kHT>::kWarps;            // consumer warps
+  constexpr int kDecStagePages = DecodeCfg<kFp8, kHT>::kStagePages;
   constexpr int kStages = L::kStages;
   constexpr int kKSteps = D / 16;     // MMA K-steps of K.Q^T
 

@@ -48,22 +48,22 @@ frt_status device_info(DeviceInfo** out) {
       di.sm_count = sms;
       if (cudaFuncSetAttribute(decode_splitkv_kernel<128, 1, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<128>::kBytes) != cudaSuccess ||
+                               DecodeSmem<128, false, 1>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(decode_splitkv_kernel<128, 2, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<128>::kBytes) != cudaSuccess ||
+                               DecodeSmem<128, false, 2>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(decode_splitkv_kernel<64, 1, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<64>::kBytes) != cudaSuccess ||
+                               DecodeSmem<64, false, 1>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(decode_splitkv_kernel<64, 2, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<64>::kBytes) != cudaSuccess ||
+                               DecodeSmem<64, false, 2>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(decode_splitkv_kernel<128, 1, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<128, true>::kBytes) != cudaSuccess ||
+                               DecodeSmem<128, true, 1>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(decode_splitkv_kernel<128, 2, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeSmem<128, true>::kBytes) != cudaSuccess ||
+                               DecodeSmem<128, true, 2>::kBytes) != cudaSuccess ||
           cudaFuncSetAttribute(prefill_kernel<128, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrefillSmem<128>::kBytes) != cudaSuccess ||
@@ -266,13 +266,32 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
 
   // one 8-head tile per segment when a KV head serves at most 8 query heads
   const bool one_tile = g <= 8;
-  const size_t smem = fp8 ? DecodeSmem<128, true>::kBytes
-                          : (D == 128) ? DecodeSmem<128>::kBytes : DecodeSmem<64>::kBytes;
-  auto* kernel =
-      fp8 ? (one_tile ? decode_splitkv_kernel<128, 1, true> : decode_splitkv_kernel<128, 2, true>)
-      : (D == 128) ? (one_tile ? decode_splitkv_kernel<128, 1, false> : decode_splitkv_kernel<128, 2, false>)
-                   : (one_tile ? decode_splitkv_kernel<64, 1, false> : decode_splitkv_kernel<64, 2, false>);
-  if (launch_pdl(kernel, dim3(parts), dim3(kDecThreads), smem, stream, tk, tv, p) != cudaSuccess)
+  // kernel, its shared memory and block size for this cache type and head tiling
+  void (*kernel)(CUtensorMap, CUtensorMap, DecodeParams) = nullptr;
+  size_t smem = 0;
+  int threads = 0;
+  auto pick = [&](auto k, size_t bytes, int nthreads) {
+    kernel = k;
+    smem = bytes;
+    threads = nthreads;
+  };
+  if (fp8) {
+    if (one_tile)
+      pick(decode_splitkv_kernel<128, 1, true>, DecodeSmem<128, true, 1>::kBytes, DecodeCfg<true, 1>::kThreads);
+    else
+      pick(decode_splitkv_kernel<128, 2, true>, DecodeSmem<128, true, 2>::kBytes, DecodeCfg<true, 2>::kThreads);
+  } else if (D == 128) {
+    if (one_tile)
+      pick(decode_splitkv_kernel<128, 1, false>, DecodeSmem<128, false, 1>::kBytes, DecodeCfg<false, 1>::kThreads);
+    else
+      pick(decode_splitkv_kernel<128, 2, false>, DecodeSmem<128, false, 2>::kBytes, DecodeCfg<false, 2>::kThreads);
+  } else {
+    if (one_tile)
+      pick(decode_splitkv_kernel<64, 1, false>, DecodeSmem<64, false, 1>::kBytes, DecodeCfg<false, 1>::kThreads);
+    else
+      pick(decode_splitkv_kernel<64, 2, false>, DecodeSmem<64, false, 2>::kBytes, DecodeCfg<false, 2>::kThreads);
+  }
+  if (launch_pdl(kernel, dim3(parts), dim3(threads), smem, stream, tk, tv, p) != cudaSuccess)
     return FRT_ERR_CUDA;
 
   // The merge of split segments: its CTAs are scheduled while the kernel
