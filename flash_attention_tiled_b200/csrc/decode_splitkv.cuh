@@ -39,14 +39,16 @@
 namespace frt {
 
 constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
-constexpr int kDecPagesPerWarp = 2;   // pages a consumer warp takes per stage
-// Consumer warps per CTA (a power of two): 4 for an FP8 cache with one 8-head
-// tile (a stage of 8 FP8 pages is 32 KB, and the consumers, not HBM, set the
-// pace), else 2.
+// Consumer warps per CTA (a power of two) and the pages each takes per
+// stage.  With one 8-head tile the consumers, not HBM, set the pace with two
+// warps, so there are four: two pages each for the FP8 cache (a stage of 8
+// FP8 pages is 32 KB), one each for bf16 (4 pages, 32 KB).  Otherwise two
+// warps of two pages.
 template <bool kFp8, int kHT>
 struct DecodeCfg {
-  static constexpr int kWarps = (kFp8 && kHT == 1) ? 4 : 2;
-  static constexpr int kStagePages = kWarps * kDecPagesPerWarp;
+  static constexpr int kWarps = (kHT == 1) ? 4 : 2;
+  static constexpr int kPagesPerWarp = (kHT == 1 && !kFp8) ? 1 : 2;
+  static constexpr int kStagePages = kWarps * kPagesPerWarp;
   static constexpr int kThreads = 32 * (kWarps + 1);
 };
 // Up to two CTAs share an SM: two independent TMA rings per SM keep more
@@ -157,6 +159,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   using L = DecodeSmem<D, kFp8, kHT>;
   constexpr int kDecWarps = DecodeCfg<kFp8, kHT>::kWarps;            // consumer warps
   constexpr int kDecStagePages = DecodeCfg<kFp8, kHT>::kStagePages;
+  constexpr int kPPW = DecodeCfg<kFp8, kHT>::kPagesPerWarp;            // pages per warp per stage
   constexpr int kStages = L::kStages;
   constexpr int kKSteps = D / 16;     // MMA K-steps of K.Q^T
 
@@ -386,25 +389,25 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int pb = pc.pg0; pb < pc.pg1; pb += kDecStagePages) {
       ok = mbar_wait_warp(&full_bar[stage], phase, &abort_flag);
       if (!ok) break;
-      const int page_a = pb + kDecPagesPerWarp * cw;     // this warp's two pages
+      const int page_a = pb + kPPW * cw;     // this warp's first page
       int valid[2];
       valid[0] = page_a < pc.pg1 ? min(kDecPage, len - page_a * kDecPage) : 0;
-      valid[1] = page_a + 1 < pc.pg1 ? min(kDecPage, len - (page_a + 1) * kDecPage) : 0;
+      valid[1] = (kPPW == 2 && page_a + 1 < pc.pg1) ? min(kDecPage, len - (page_a + 1) * kDecPage) : 0;
       if (valid[0] > 0) {
         const int npg = valid[1] > 0 ? 2 : 1;
         const uint32_t base = ring_u32 + stage * L::kStageBytes +
-                              kDecPagesPerWarp * cw * 2 * L::kPageBytes;
+                              kPPW * cw * 2 * L::kPageBytes;
         // ---- S^T = K.Q^T per page (fragment loads of a page issued first)
         float sacc[2][kHT][4];
 #pragma unroll
-        for (int pg = 0; pg < 2; ++pg)
+        for (int pg = 0; pg < kPPW; ++pg)
 #pragma unroll
           for (int ht = 0; ht < kHT; ++ht) sacc[pg][ht][0] = sacc[pg][ht][1] = sacc[pg][ht][2] = sacc[pg][ht][3] = 0.f;
         {
           const int mi = lane >> 3, j = lane & 7;
           const int tok = (mi & 1) * 8 + j;
 #pragma unroll
-          for (int pg = 0; pg < 2; ++pg) {
+          for (int pg = 0; pg < kPPW; ++pg) {
             if (pg < npg) {
               const uint32_t kbase = base + pg * 2 * L::kPageBytes;
               if constexpr (kFp8) {
@@ -453,7 +456,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int ht = 0; ht < kHT; ++ht) {
           float sc[2][4];
 #pragma unroll
-          for (int pg = 0; pg < 2; ++pg)
+          for (int pg = 0; pg < kPPW; ++pg)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int tok = r8 + (i >> 1) * 8;
@@ -462,7 +465,8 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           float e[2][4];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            float mx = fmaxf(fmaxf(sc[0][hh], sc[0][2 + hh]), fmaxf(sc[1][hh], sc[1][2 + hh]));
+            float mx = fmaxf(sc[0][hh], sc[0][2 + hh]);
+            if (kPPW == 2) mx = fmaxf(mx, fmaxf(sc[1][hh], sc[1][2 + hh]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -470,7 +474,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             alpha[ht][hh] = fast_exp2(m_run[ht][hh] - m_new);   // 0 on the first step
             m_run[ht][hh] = m_new;
 #pragma unroll
-            for (int pg = 0; pg < 2; ++pg) {
+            for (int pg = 0; pg < kPPW; ++pg) {
               e[pg][hh] = fast_exp2(sc[pg][hh] - m_new);
               e[pg][2 + hh] = fast_exp2(sc[pg][2 + hh] - m_new);
             }
@@ -481,7 +485,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             le_run[ht][hh] *= alpha[ht][hh];
           }
 #pragma unroll
-          for (int pg = 0; pg < 2; ++pg) {
+          for (int pg = 0; pg < kPPW; ++pg) {
             // rows r8 (lo) and r8+8 (hi) of S^T as 16-bit pairs (heads 2qc,
             // 2qc+1): bf16, or f16 for the FP8 cache.  O is normalised by the
             // rounded weights that feed P.V; the LSE uses the exact ones
@@ -530,7 +534,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int mi = lane >> 3, j = lane & 7;
           const int tok = (mi & 1) * 8 + j;
 #pragma unroll
-          for (int pg = 0; pg < 2; ++pg) {
+          for (int pg = 0; pg < kPPW; ++pg) {
             if (pg < npg) {
               const uint32_t vbase = base + pg * 2 * L::kPageBytes + L::kPageBytes;
               uint32_t vr[kMT / 2][4];
@@ -567,7 +571,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int mi = lane >> 3, j = lane & 7;
           const int tok = (mi >> 1) * 8 + j;
 #pragma unroll
-          for (int pg = 0; pg < 2; ++pg) {
+          for (int pg = 0; pg < kPPW; ++pg) {
             if (pg < npg) {
               const uint32_t vbase = base + pg * 2 * L::kPageBytes + L::kPageBytes;
               uint32_t vf[kMT][4];
