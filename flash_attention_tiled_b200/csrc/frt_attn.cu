@@ -315,32 +315,47 @@ struct PagedKV {
   int max_pages, num_pages;
 };
 
+// Element strides of a [B, H, S, D] tensor's batch, head and token
+// dimensions (d is contiguous).
+struct TokStrides {
+  long long b, h, t;
+};
+
 frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
-                          float scale, cudaStream_t stream, const PagedKV* paged = nullptr) {
+                          float scale, cudaStream_t stream, const PagedKV* paged = nullptr,
+                          const TokStrides* strides = nullptr /* q, k, v, o; null: contiguous */) {
   DeviceInfo* di = nullptr;
   frt_status st = device_info(&di);
   if (st != FRT_OK) return st;
   if (!di->prefill_ok) return FRT_ERR_UNSUPPORTED;
   const int n_blocks = (Sq + kPfRows - 1) / kPfRows;
   if (n_blocks > 65535) return FRT_ERR_UNSUPPORTED;
+  // Q, O (and contiguous K, V): 4D maps (d, token, head, batch) with the
+  // tensors' own strides, one 128-row box per column half
   CUtensorMap tq, tk, tv, to;
-  const uint32_t box[3] = {64, (uint32_t)kPfBM, 1};
-  const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * Hq};
-  const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
-  if (!make_tmap(&tq, q, 3, qdims, qstr, box) || !make_tmap(&to, o, 3, qdims, qstr, box))
-    return FRT_ERR_CUDA;
+  const TokStrides q_c{(long long)Hq * Sq * D, (long long)Sq * D, D};
+  const TokStrides k_c{(long long)Hkv * Skv * D, (long long)Skv * D, D};
+  const TokStrides& qs = strides ? strides[0] : q_c;
+  const TokStrides& ks = strides ? strides[1] : k_c;
+  const TokStrides& vs = strides ? strides[2] : k_c;
+  const TokStrides& os = strides ? strides[3] : q_c;
+  const uint32_t box[4] = {64, (uint32_t)kPfBM, 1, 1};
+  auto map4 = [&](CUtensorMap* m, const void* base, int S, int H, int Bn, const TokStrides& st) {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S, (uint64_t)H, (uint64_t)Bn};
+    const uint64_t str[3] = {(uint64_t)st.t * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
+    return make_tmap(m, base, 4, dims, str, box);
+  };
+  if (!map4(&tq, q, Sq, Hq, B, qs) || !map4(&to, o, Sq, Hq, B, os)) return FRT_ERR_CUDA;
   if (paged == nullptr) {
-    // With Skv == 0 every tile has no key tile to visit (o = 0, lse = -inf);
-    // the K/V maps then only need to be valid descriptors, never read.
-    const void* kb = Skv > 0 ? k : q;
-    const void* vb = Skv > 0 ? v : q;
-    const int skv_map = Skv > 0 ? Skv : 1;
-    const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)skv_map,
-                               (uint64_t)(Skv > 0 ? B * Hkv : 1)};
-    const uint64_t kstr[2] = {(uint64_t)D * 2, (uint64_t)skv_map * D * 2};
-    if (!make_tmap(&tk, kb, 3, kdims, kstr, box) || !make_tmap(&tv, vb, 3, kdims, kstr, box))
-      return FRT_ERR_CUDA;
+    if (Skv > 0) {
+      if (!map4(&tk, k, Skv, Hkv, B, ks) || !map4(&tv, v, Skv, Hkv, B, vs)) return FRT_ERR_CUDA;
+    } else {
+      // With Skv == 0 every tile has no key tile to visit (o = 0, lse =
+      // -inf); the K/V maps then only need to be valid descriptors, never read.
+      const TokStrides one{D, D, D};
+      if (!map4(&tk, q, 1, 1, 1, one) || !map4(&tv, q, 1, 1, 1, one)) return FRT_ERR_CUDA;
+    }
   } else {
     // page pool as rows of D: one 16-row box per page and column half
     const uint64_t kdims[2] = {(uint64_t)D, (uint64_t)paged->num_pages * Hkv * 16};
@@ -527,6 +542,39 @@ frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
                          Hq, Hkv, D, scale, 0, workspace, workspace_bytes, stream);
   }
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream);
+}
+
+frt_status frt_attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
+                                float scale, const int64_t* q_strides, const int64_t* k_strides,
+                                const int64_t* v_strides, const int64_t* o_strides,
+                                cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Skv < 0 ||
+      (causal != 0 && causal != 1) || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)B * Hq * Sq >= (1ull << 31) || (uint64_t)B * Hkv * Skv >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
+  if (q_strides == nullptr || k_strides == nullptr || v_strides == nullptr || o_strides == nullptr)
+    return FRT_ERR_INVALID_ARG;
+  TokStrides st[4];
+  const int64_t* src[4] = {q_strides, k_strides, v_strides, o_strides};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 3; ++j) {
+      // every step of a TMA walk is a multiple of 16 bytes (8 bf16)
+      const int64_t x = src[i][j];
+      if (x <= 0 || x % 8 != 0 || x >= (1ll << 38)) return FRT_ERR_INVALID_ARG;
+    }
+    st[i] = TokStrides{src[i][0], src[i][1], src[i][2]};
+  }
+  if (B == 0 || Sq == 0) return FRT_OK;
+  if (q == nullptr || o == nullptr || (Skv > 0 && (k == nullptr || v == nullptr)))
+    return FRT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FRT_ERR_INVALID_ARG;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream, nullptr,
+                        st);
 }
 
 frt_status frt_attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,

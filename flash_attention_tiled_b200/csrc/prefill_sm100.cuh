@@ -132,7 +132,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int blk = p.causal ? (p.n_blocks - 1 - (int)blockIdx.y) : (int)blockIdx.y;
   const int b = bh / p.Hq, hq = bh % p.Hq;
   const int kvh = hq / p.g;
-  const int kv_row = b * p.Hkv + kvh;        // z coordinate in the contiguous K/V maps
+  // Q, O, K and V maps are 4D (d, token, head, batch), so any strides work
   const int q_blk = blk * kPfRows;           // first query row of tile A
   // this sequence's chunk (query) length and context (key) length
   int sq_b = p.Sq, skv_b = p.Skv;
@@ -190,8 +190,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int t = 0; t < kPfTiles; ++t)
 #pragma unroll
           for (int h = 0; h < kHalves; ++h)
-            tma_load_3d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
-                        q_blk + t * kPfBM, bh);
+            tma_load_4d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
+                        q_blk + t * kPfBM, hq, b);
       }
       int slot = 0;
       uint32_t phase = 0;
@@ -206,8 +206,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_arrive_expect_tx(&ring_full[slot], L::kTileBytes);
 #pragma unroll
             for (int h = 0; h < kHalves; ++h)
-              tma_load_3d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN,
-                          kv_row);
+              tma_load_4d(dst + h * L::kHalfBytes, tm, &ring_full[slot], h * 64, j * kPfBN, kvh,
+                          b);
           }
         } else {
           // eight 16-token pages per key tile, each fetched through the block
@@ -516,7 +516,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const bool stop = bar_sync_or(1 + t, 128, !ok || abort_flag);
     if (!stop && quarter == 0 && lane == 0 && q0 < p.Sq) {
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h) tma_store_3d(&tm_o, so + h * L::kHalfBytes, h * 64, q0, bh);
+      for (int h = 0; h < kHalves; ++h)
+        tma_store_4d(&tm_o, so + h * L::kHalfBytes, h * 64, q0, hq, b);
       tma_store_commit();
       tma_store_wait_all();
     }

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
 EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
-           "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8",
+           "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8", "frt_attn_fwd_strided",
            "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
            "frt_debug_fp8_decode", "frt_version")
 
@@ -50,6 +50,7 @@ def _load() -> ctypes.CDLL:
     lib.frt_attn_decode_paged_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I,
                                               P, Z, P]
     lib.frt_debug_fp8_decode.argtypes = [P, P, I, P]
+    lib.frt_attn_fwd_strided.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, P, P]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = ctypes.c_int
     lib.frt_version.restype = ctypes.c_char_p
@@ -203,6 +204,37 @@ def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), ps, P, _ptr(out), _ptr(lse), B, Hq, Hkv, D, scale,
         num_splits, _ptr(ws), ctypes.byref(need), stream))
+    return out, lse
+
+
+def _strides3(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or t.dim() != 4:
+        raise ValueError(f"{name} must be a 4-dim bf16 tensor [B, H, S, D]")
+    if t.stride(3) != 1:
+        raise ValueError(f"{name}: the last (head-dim) axis must be contiguous")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                     scale: float | None = None, out: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, return_lse: bool = True):
+    """attn_fwd for views in any layout: q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D] with
+    any batch/head/token strides (multiples of 8 elements) and a contiguous
+    last axis, e.g. views into a fused QKV tensor.  `out` may be a strided
+    view too (default: a new contiguous [B,Hq,Sq,D])."""
+    qs, ks, vs = _strides3(q, "q"), _strides3(k, "k"), _strides3(v, "v")
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, D), dtype=q.dtype, device=q.device)
+    os_ = _strides3(out, "out")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _check("frt_attn_fwd_strided", _lib.frt_attn_fwd_strided(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, int(causal), scale,
+        qs, ks, vs, os_, _stream(q.device)))
     return out, lse
 
 

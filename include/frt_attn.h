@@ -213,6 +213,32 @@ FRT_API frt_status frt_attn_decode_paged_noalloc(const void* q, const void* k_pa
                                                  cudaStream_t stream);
 
 /*
+ * frt_attn_fwd_strided -- frt_attn_fwd for tensors in any strided layout, e.g.
+ * views into a fused QKV projection output [B, S, 3, H, D] or a [B, S, H, D]
+ * cache, with no copy.  The Triton sketch of the "Real-time inference
+ * optimisation" page (section "Flash Attention optimisation") takes a
+ * stride per dimension of Q, K, V and O for the same reason.
+ *   q, k, v, o  bf16; element (b, h, s, d) of a tensor is at
+ *               base + b*strides[0] + h*strides[1] + s*strides[2] + d
+ *               (d contiguous), with shapes [B,Hq,Sq,D], [B,Hkv,Skv,D] x2,
+ *               [B,Hq,Sq,D]
+ *   *_strides   host arrays of three int64 element strides (batch, head,
+ *               token); each a positive multiple of 8 (the copy engine
+ *               steps in 16-byte units), below 2^38
+ *   lse         [B,Hq,Sq] fp32 contiguous, may be NULL
+ * Every other argument as frt_attn_fwd.  All Sq (1 included) run the tiled
+ * tensor-core kernel; for single-token decode over a contiguous cache
+ * frt_attn_fwd (or a paged cache) is faster.  o must not overlap q, k or v,
+ * and its strides must not map two elements to one address.
+ */
+FRT_API frt_status frt_attn_fwd_strided(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int Hq, int Hkv, int Sq, int Skv,
+                                        int D, int causal, float scale,
+                                        const int64_t* q_strides, const int64_t* k_strides,
+                                        const int64_t* v_strides, const int64_t* o_strides,
+                                        cudaStream_t stream);
+
+/*
  * frt_attn_decode_paged_fp8 -- frt_attn_decode_paged over an FP8 KV cache.
  * The FasterTransformer read-through (pptc.cn) keeps the KV cache quantised
  * and dequantises it before use (section 3.3, an int8 KV cache) and enables

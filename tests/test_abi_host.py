@@ -135,3 +135,27 @@ def test_decode_fp8_workspace_query_matches_bf16():
 def test_debug_fp8_decode_rejects():
     assert frt.lib().frt_debug_fp8_decode(NULL, NULL, -1, NULL) == 1
     assert frt.lib().frt_debug_fp8_decode(NULL, NULL, 0, NULL) == 0
+
+
+def _strided(B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64, causal=0, scale=0.125, qs=(512, 256, 64),
+             ks=(512, 256, 64), vs=(512, 256, 64), os_=(512, 256, 64)):
+    arr = lambda t: None if t is None else (ctypes.c_int64 * 3)(*t)
+    return frt.lib().frt_attn_fwd_strided(NULL, NULL, NULL, NULL, NULL, B, Hq, Hkv, Sq, Skv, D,
+                                          causal, scale, arr(qs), arr(ks), arr(vs), arr(os_), NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), 1),
+    (dict(D=96), 2),
+    (dict(qs=(512, 256, 60)), 1),         # a token step that is not 16 bytes
+    (dict(ks=(512, -256, 64)), 1),
+    (dict(vs=(0, 256, 64)), 1),
+    (dict(os_=None), 1),
+    (dict(scale=-1.0), 1),
+])
+def test_fwd_strided_rejects(kw, code):
+    assert _strided(**kw) == code
+
+
+def test_fwd_strided_empty_is_a_noop():
+    assert _strided(B=0) == 0 and _strided(Sq=0) == 0

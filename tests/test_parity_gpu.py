@@ -360,6 +360,54 @@ def test_fp8_decode_deterministic(frt):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# --------------------------------------------------------- strided layouts
+STRIDED_CASES = [  # B, Hq, Hkv, Sq, Skv, D, causal, fused
+    (2, 4, 4, 300, 300, 128, True, "qkv"),     # fused [B,S,3,H,D] projection output, MHA
+    (1, 8, 2, 257, 257, 64, True, "gqa"),      # fused [B,S,Hq+2Hkv,D], GQA
+    (2, 4, 2, 130, 577, 128, False, "bshd"),   # cross attention, [B,S,H,D] tensors
+    (3, 8, 2, 1, 999, 128, False, "bshd"),     # single-token rows, tile kernel
+]
+
+
+def _strided_inputs(case, seed):
+    B, Hq, Hkv, Sq, Skv, D, causal, fused = case
+    g = torch.Generator().manual_seed(seed)
+    rnd = lambda *shape: torch.randn(*shape, generator=g).to(torch.bfloat16).cuda()
+    if fused == "qkv":
+        qkv = rnd(B, Sq, 3, Hq, D)
+        q, k, v = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    elif fused == "gqa":
+        x = rnd(B, Sq, Hq + 2 * Hkv, D)
+        q = x[:, :, :Hq].permute(0, 2, 1, 3)
+        k = x[:, :, Hq:Hq + Hkv].permute(0, 2, 1, 3)
+        v = x[:, :, Hq + Hkv:].permute(0, 2, 1, 3)
+    else:
+        q = rnd(B, Sq, Hq, D).permute(0, 2, 1, 3)
+        k = rnd(B, Skv, Hkv, D).permute(0, 2, 1, 3)
+        v = rnd(B, Skv, Hkv, D).permute(0, 2, 1, 3)
+    return q, k, v
+
+
+@pytest.mark.parametrize("case", STRIDED_CASES, ids=str)
+def test_strided_layouts(frt, case):
+    B, Hq, Hkv, Sq, Skv, D, causal, fused = case
+    q, k, v = _strided_inputs(case, seed=Sq + Skv)
+    assert Sq == 1 or not q.is_contiguous()   # (a one-token view counts as contiguous)
+    out_buf = torch.full((B, Sq, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = out_buf.permute(0, 2, 1, 3)                    # a strided output view
+    o, lse = frt.attn_fwd_strided(q, k, v, causal=causal, out=out)
+    torch.cuda.synchronize()
+    qc, kc, vc = q.contiguous(), k.contiguous(), v.contiguous()
+    o_ref, lse_ref = oracle.attn_fwd(qc.cpu(), kc.cpu(), vc.cpu(), causal, 1 / math.sqrt(D))
+    _compare(out, o_ref, lse, lse_ref, f"strided {case}")
+    if Sq > 1:
+        # the same tile kernel on contiguous copies: bit-identical
+        o2, l2 = frt.attn_fwd(qc, kc, vc, causal=causal)
+        torch.cuda.synchronize()
+        assert torch.equal(out.contiguous(), o2) and torch.equal(lse, l2)
+    _no_device_error(frt)
+
+
 # ------------------------------------------------------------------- merge
 @pytest.mark.parametrize("S,B,Hq,D,empty", [(1, 2, 8, 128, 0.0), (5, 3, 16, 128, 0.3),
                                             (37, 1, 32, 128, 0.0), (4, 2, 4, 64, 0.5)])
