@@ -175,9 +175,12 @@ class Step:
     """The four calls of one step, with inputs resident on the device."""
 
     ALL = ("prefill", "paged", "long", "contig")
+    # the paged workloads with their cache stored as e4m3 (not part of the
+    # configured step; --calls may name them, e.g. for a profile)
+    FP8 = ("paged_fp8", "long_fp8")
     # kernels each call launches: prefill_kernel; decode_splitkv_kernel then
     # decode_merge_kernel
-    LAUNCHES = {"prefill": 1, "paged": 2, "long": 2, "contig": 2}
+    LAUNCHES = {"prefill": 1, "paged": 2, "long": 2, "contig": 2, "paged_fp8": 2, "long_fp8": 2}
 
     def __init__(self, device, names=ALL):
         from flash_attention_tiled_b200 import frt
@@ -189,18 +192,30 @@ class Step:
         self.w_pg = W["paged_gqa_decode_b4"]
         self.w_lg = W["long_splitkv_decode_256k"]
         self.w_ct = W["gqa_decode_4k"]
-        wl = {"prefill": self.w_pf, "paged": self.w_pg, "long": self.w_lg, "contig": self.w_ct}
-        self.host = {n: inputs.make(wl[n]) for n in self.NAMES}
+        wl = {"prefill": self.w_pf, "paged": self.w_pg, "long": self.w_lg, "contig": self.w_ct,
+              "paged_fp8": self.w_pg, "long_fp8": self.w_lg}
+
+        def make(n):
+            w = wl[n]
+            if n in Step.FP8:
+                return inputs.paged_fp8(w.B, w.Hq, w.Hkv, w.D, len_range=w.len_range,
+                                        page_size=w.page_size, seed=w.seed)
+            return inputs.make(w)
+
+        self.host = {n: make(n) for n in self.NAMES}
         self.d = {k: {n: (t.to(device) if isinstance(t, torch.Tensor) else t)
                       for n, t in v.items()} for k, v in self.host.items()}
         if "paged" in self.NAMES:
             self.tokens_pg = int(self.host["paged"]["seq_lens"].sum())
         if "long" in self.NAMES:
             self.tokens_lg = int(self.host["long"]["seq_lens"].sum())
+        self.tokens = {n: int(self.host[n]["seq_lens"].sum()) for n in self.NAMES
+                       if n in Step.FP8}
         # outputs, allocated once
         shapes = {"prefill": (self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq),
                   "paged": (self.w_pg.B, self.w_pg.Hq), "long": (self.w_lg.B, self.w_lg.Hq),
-                  "contig": (self.w_ct.B, self.w_ct.Hq, 1)}
+                  "contig": (self.w_ct.B, self.w_ct.Hq, 1),
+                  "paged_fp8": (self.w_pg.B, self.w_pg.Hq), "long_fp8": (self.w_lg.B, self.w_lg.Hq)}
         self.out = {n: (torch.empty_like(self.d[n]["q"]), torch.empty(shapes[n], device=device))
                     for n in self.NAMES}
 
@@ -212,6 +227,10 @@ class Step:
             f.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=self.w_pf.scale, out=o, lse=l)
         elif name == "contig":
             f.attn_fwd(d["q"], d["k"], d["v"], causal=False, scale=self.w_ct.scale, out=o, lse=l)
+        elif name in Step.FP8:
+            w = self.w_pg if name == "paged_fp8" else self.w_lg
+            f.attn_decode_paged_fp8(d["q"], d["k_pages"], d["v_pages"], d["k_scale"], d["v_scale"],
+                                    d["block_table"], d["seq_lens"], scale=w.scale, out=o, lse=l)
         else:
             w = self.w_pg if name == "paged" else self.w_lg
             f.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"],
@@ -230,6 +249,11 @@ class Step:
             elif n == "long":
                 out[n] = (decode_flops(self.w_lg.Hq, 128, self.tokens_lg),
                           decode_bytes(1, self.w_lg.Hq, self.w_lg.Hkv, 128, self.tokens_lg))
+            elif n in Step.FP8:
+                w, t = (self.w_pg if n == "paged_fp8" else self.w_lg), self.tokens[n]
+                # one byte per cached K/V element
+                out[n] = (decode_flops(w.Hq, 128, t),
+                          decode_bytes(w.B, w.Hq, w.Hkv, 128, t) - 2.0 * t * w.Hkv * 128)
             else:
                 out[n] = (decode_flops(self.w_ct.Hq, 128, self.w_ct.Skv),
                           decode_bytes(1, self.w_ct.Hq, self.w_ct.Hkv, 128, self.w_ct.Skv))
@@ -341,6 +365,13 @@ def run_ours(args, rank, world, local_rank):
     t_flush = graph_ms(g_flush)
     per_call_ms = {n: max(graph_ms(g_call[n]) - t_flush, 1e-6) / R for n in names}
 
+    # ---- the FP8-cache decode on the two paged workloads (not part of the
+    # step: the step is the configured workload), timed the same way
+    extras = None
+    if not args.no_extras:
+        extras = run_fp8_extras(device, stream, flush, R, graph_ms, t_flush)
+        extras.update(run_tile_extras(device, stream, flush, R, graph_ms, t_flush))
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -375,7 +406,9 @@ def run_ours(args, rank, world, local_rank):
     # call's time also holds its small merge kernel (timed together, so the
     # streaming kernel's fraction is if anything understated).
     kernel_of = {"prefill": "prefill_kernel<128>", "paged": "decode_splitkv_kernel<128>",
-                 "long": "decode_splitkv_kernel<128>", "contig": "decode_splitkv_kernel<128>"}
+                 "long": "decode_splitkv_kernel<128>", "contig": "decode_splitkv_kernel<128>",
+                 "paged_fp8": "decode_splitkv_kernel<128> (e4m3 cache)",
+                 "long_fp8": "decode_splitkv_kernel<128> (e4m3 cache)"}
     per_kernel = {}
     for n in names:
         k = kernel_of[n]
@@ -428,6 +461,7 @@ def run_ours(args, rank, world, local_rank):
                          "before each call (2x L2 size written, then another 2x L2 "
                          "read so the written lines are clean)"},
         "calls": calls,
+        "extras": extras,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -435,6 +469,97 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary(),
     }
     return line
+
+
+def run_fp8_extras(device, stream, flush, R, graph_ms, t_flush):
+    """Per-call µs and GB/s of frt_attn_decode_paged_fp8 on the paged B4 and
+    256k workloads with the cache stored as e4m3 (per-KV-head scales); L2
+    flushed before each call as for the step's calls."""
+    from flash_attention_tiled_b200 import frt
+    peaks, _ = load_peaks()
+    res = {}
+    for name, wname in (("paged_fp8", "paged_gqa_decode_b4"), ("long_fp8", "long_splitkv_decode_256k")):
+        w = inputs.WORKLOADS[wname]
+        x = inputs.paged_fp8(w.B, w.Hq, w.Hkv, w.D, len_range=w.len_range, page_size=w.page_size,
+                             seed=w.seed)
+        d = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        o = torch.empty_like(d["q"])
+        lse = torch.empty((w.B, w.Hq), device=device)
+
+        def call():
+            frt.attn_decode_paged_fp8(d["q"], d["k_pages"], d["v_pages"], d["k_scale"],
+                                      d["v_scale"], d["block_table"], d["seq_lens"],
+                                      scale=w.scale, out=o, lse=lse)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(R):
+                flush()
+                call()
+        us = max(graph_ms(g) - t_flush, 1e-6) / R * 1e3
+        tokens = int(x["seq_lens"].sum())
+        # one byte per cached K/V element, plus q, o and lse
+        nbytes = 2.0 * tokens * w.Hkv * w.D + w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4
+        gbs = nbytes / us * 1e-3
+        res[name] = {"us": round(us, 2), "gbs": round(gbs, 1), "bytes": nbytes, "bound": "hbm",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "cache": "e4m3 codes, per-KV-head fp32 scale", "workload": wname}
+        del g, d, x
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_tile_extras(device, stream, flush, R, graph_ms, t_flush):
+    """Per-call µs and TFLOP/s of the tile kernel on two more shapes: cross
+    attention (1024 queries over 4096 keys, non-causal, GQA 32/8, D 128) and
+    the Llama-3-8B causal prefill read through views of a fused
+    [B, S, Hq + 2 Hkv, D] projection output (frt_attn_fwd_strided)."""
+    from flash_attention_tiled_b200 import frt
+    peaks, _ = load_peaks()
+    gen = torch.Generator("cpu").manual_seed(2024)
+    res = {}
+    w = inputs.WORKLOADS["llama3_8b_prefill_4k"]
+    cases = []
+    # cross attention: contiguous [B,H,S,D] tensors
+    Sq, Skv = 1024, 4096
+    q = torch.randn(1, 32, Sq, 128, generator=gen).to(torch.bfloat16).to(device)
+    k = torch.randn(1, 8, Skv, 128, generator=gen).to(torch.bfloat16).to(device)
+    v = torch.randn(1, 8, Skv, 128, generator=gen).to(torch.bfloat16).to(device)
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 32, Sq), device=device)
+    cases.append(("cross_attn", lambda: frt.attn_fwd(q, k, v, causal=False, out=o, lse=lse),
+                  4.0 * 128 * Sq * Skv * 32, "B1 Hq32 Hkv8 Sq1024 Skv4096 D128, non-causal"))
+    # the Llama-3-8B prefill from a fused projection output
+    x = torch.randn(w.B, w.Sq, w.Hq + 2 * w.Hkv, w.D, generator=gen).to(torch.bfloat16).to(device)
+    qs = x[:, :, :w.Hq].permute(0, 2, 1, 3)
+    ks = x[:, :, w.Hq:w.Hq + w.Hkv].permute(0, 2, 1, 3)
+    vs = x[:, :, w.Hq + w.Hkv:].permute(0, 2, 1, 3)
+    os_ = torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16, device=device).permute(0, 2, 1, 3)
+    lse2 = torch.empty((w.B, w.Hq, w.Sq), device=device)
+    cases.append(("prefill_strided",
+                  lambda: frt.attn_fwd_strided(qs, ks, vs, causal=True, scale=w.scale, out=os_,
+                                               lse=lse2),
+                  prefill_flops(w), "Llama-3-8B causal 4k, Q/K/V/O as views of [B,S,H,D] buffers"))
+    for name, call, flop, desc in cases:
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(R):
+                flush()
+                call()
+        us = max(graph_ms(g) - t_flush, 1e-6) / R * 1e3
+        tf = flop / us * 1e-6
+        res[name] = {"us": round(us, 2), "tflops": round(tf, 1), "flop": flop, "bound": "tensor",
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "workload": desc}
+        del g
+    return res
 
 
 def run_e2e(st: Step, args, device):
@@ -565,12 +690,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the FP8-cache decode, cross-attention and strided-prefill "
+                         "measurements")
     ap.add_argument("--calls", default=",".join(Step.ALL),
                     help="comma-separated subset of the step's calls (profiling runs)")
     args = ap.parse_args()
     args.calls = tuple(c for c in args.calls.split(",") if c)
-    if not set(args.calls) <= set(Step.ALL):
-        ap.error(f"--calls must be a subset of {Step.ALL}")
+    if not set(args.calls) <= set(Step.ALL + Step.FP8):
+        ap.error(f"--calls must be a subset of {Step.ALL + Step.FP8}")
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
