@@ -4,7 +4,8 @@ One step = one pass of every operation on the path over its own seeded,
 HBM-resident synthetic input:
   prefill   Llama-3-8B-shaped causal prefill   B1 Hq32 Hkv8 S4096 D128  (frt_attn_fwd)
   paged     paged GQA decode                   B4 Hq64 Hkv8 D128 ps16, lens U[1024,32768]
-                                               (frt_attn_decode_paged, fused LSE merge)
+                                               (frt_attn_decode_paged: streaming kernel,
+                                               then the dependent LSE merge kernel)
   long      long-context split-KV decode       B1 Hq32 Hkv4 Skv262144 D128 ps16
   contig    single-token GQA decode            B1 Hq32 Hkv8 Skv4096 D128 (frt_attn_fwd, Sq=1)
 Each step's working set (~0.9 GB) exceeds the 126 MB L2, and every call's
@@ -12,7 +13,9 @@ inputs are evicted by the calls before it, so no call starts L2-warm.
 
 Prints ONE JSON line (rank 0).  `value` is whole-job steps per second; the
 per-call microseconds, TFLOP/s, GB/s and roofline fractions are under
-"calls"; "roofline" describes the dominant kernel.
+"calls"; "roofline" describes the dominant kernel; "extras" holds calls
+outside the step (the FP8-cache decode on the two paged workloads, cross
+attention, the prefill through strided views), timed the same way.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 

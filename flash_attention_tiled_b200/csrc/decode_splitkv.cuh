@@ -25,8 +25,9 @@
 // Inside a CTA (two per SM): warp 0 streams pages into a ring of
 // shared-memory stages with TMA (one 128-byte swizzled box per page and
 // matrix, one mbarrier per stage), looking pages up in the block table;
-// warps 1..W each take two pages (32 tokens) of every stage and compute
-// S^T = K.Q^T and O^T += V^T.P^T with warp-level bf16 MMAs in which a page's
+// warps 1..W (DecodeCfg) each take one or two pages of every stage and compute
+// S^T = K.Q^T and O^T += V^T.P^T with warp-level MMAs (bf16, or f16 from an
+// e4m3 cache) in which a page's
 // tokens form the M dimension of the first and the segment's query heads the
 // N dimension of both, so each K/V page is read from HBM once for all heads
 // of its group.  Scores live in the exp2 domain (scale * log2(e) folded in).
