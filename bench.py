@@ -50,14 +50,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def source_sha() -> str:
-    """Hash of the CUDA sources, to tell whether profiled counters still apply."""
+    """Hash of the CUDA sources' code (comments and whitespace removed), to tell
+    whether profiled counters still apply: a comment edit keeps them, a code
+    change retires them."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "flash_attention_tiled_b200", "csrc", "*"))):
+        if not f.endswith((".cu", ".cuh", ".h")):
+            continue
+        with open(f, encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
