@@ -360,6 +360,46 @@ def test_fp8_decode_deterministic(frt):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# -------------------------------------------------- exact special cases
+def test_single_visible_key_gives_v_exactly(frt):
+    # one key: p = 1 and l = 1, so o is that key's value row, bit for bit
+    x = inputs.dense(2, 4, 2, 3, 1, 128, seed=21)
+    d = _dev(x)
+    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=False)          # tile kernel (Sq = 3)
+    torch.cuda.synchronize()
+    g = 4 // 2
+    for h in range(4):
+        assert torch.equal(o[:, h].cpu(), x["v"][:, h // g, :1].expand(-1, 3, -1))
+    p = inputs.paged(3, 8, 2, 128, seq_lens=[1, 1, 1], seed=22)
+    dp = _dev(p)
+    o, _ = frt.attn_decode_paged(dp["q"], dp["k_pages"], dp["v_pages"], dp["block_table"],
+                                 dp["seq_lens"])
+    torch.cuda.synchronize()
+    for b in range(3):
+        phys = int(p["block_table"][b, 0])
+        for h in range(8):
+            assert torch.equal(o[b, h].cpu(), p["v_pages"][phys, h // 4, 0])
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads(frt):
+    B, Hq, Hkv, S, D = 1, 8, 2, 300, 128
+    x = inputs.dense(B, Hq, Hkv, S, S, D, seed=23)
+    d = _dev(x)
+    g = Hq // Hkv
+    k_rep, v_rep = (t.repeat_interleave(g, dim=1).contiguous() for t in (d["k"], d["v"]))
+    o1, l1 = frt.attn_fwd(d["q"], d["k"], d["v"], causal=True)
+    o2, l2 = frt.attn_fwd(d["q"], k_rep, v_rep, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)        # same per-head arithmetic
+    # decode: the head grouping changes the split plan, so compare within the bar
+    q1 = d["q"][:, :, :1].contiguous()
+    o1, l1 = frt.attn_fwd(q1, d["k"], d["v"])
+    o2, l2 = frt.attn_fwd(q1, k_rep, v_rep)
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= MAX_ABS
+    assert (l1 - l2).abs().max().item() <= LSE_ABS
+
+
 # --------------------------------------------------------- strided layouts
 STRIDED_CASES = [  # B, Hq, Hkv, Sq, Skv, D, causal, fused
     (2, 4, 4, 300, 300, 128, True, "qkv"),     # fused [B,S,3,H,D] projection output, MHA
