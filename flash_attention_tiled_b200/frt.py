@@ -92,6 +92,33 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t: torch.Tensor, name: str, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _out(t, name: str, dtype, shape, device, contiguous: bool = True):
+    """A caller-supplied output: right dtype, shape and device (the kernels
+    write exactly that many elements)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    _shape(t, name, shape)
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the inputs on {device}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(device, **tensors):
+    for name, t in tensors.items():
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, q on {device}")
+
+
 # Workspaces, one per (device, stream, shape): a call writes every word of
 # the workspace it later reads, so one buffer serves all later calls of the
 # same shape ordered on the same stream.
@@ -115,6 +142,11 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
         _need(t, n, torch.bfloat16, 4)
     B, Hq, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape
+    _shape(k, "k", (B, Hkv, Skv, D))
+    _shape(v, "v", k.shape)
+    _same_device(q.device, k=k, v=v)
+    _out(out, "out", torch.bfloat16, q.shape, q.device)
+    _out(lse, "lse", torch.float32, (B, Hq, Sq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -149,6 +181,14 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
     _need(seq_lens, "seq_lens", torch.int32, 1)
     B, Hq, D = q.shape
     P, Hkv, ps, _ = k_pages.shape
+    _shape(k_pages, "k_pages", (P, Hkv, ps, D))
+    _shape(v_pages, "v_pages", k_pages.shape)
+    _shape(block_table, "block_table", (B, block_table.shape[1]))
+    _shape(seq_lens, "seq_lens", (B,))
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens)
+    _out(out, "out", torch.bfloat16, q.shape, q.device)
+    _out(lse, "lse", torch.float32, (B, Hq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -187,6 +227,16 @@ def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch
     _need(seq_lens, "seq_lens", torch.int32, 1)
     B, Hq, D = q.shape
     P, Hkv, ps, _ = k_pages.shape
+    _shape(k_pages, "k_pages", (P, Hkv, ps, D))
+    _shape(v_pages, "v_pages", k_pages.shape)
+    _shape(k_scale, "k_scale", (Hkv,))
+    _shape(v_scale, "v_scale", (Hkv,))
+    _shape(block_table, "block_table", (B, block_table.shape[1]))
+    _shape(seq_lens, "seq_lens", (B,))
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, k_scale=k_scale, v_scale=v_scale,
+                 block_table=block_table, seq_lens=seq_lens)
+    _out(out, "out", torch.bfloat16, q.shape, q.device)
+    _out(lse, "lse", torch.float32, (B, Hq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -225,6 +275,14 @@ def attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: 
     qs, ks, vs = _strides3(q, "q"), _strides3(k, "k"), _strides3(v, "v")
     B, Hq, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape
+    _shape(k, "k", (B, Hkv, Skv, D))
+    _shape(v, "v", k.shape)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not t.is_cuda:
+            raise TypeError(f"{n} must be a CUDA tensor")
+    _same_device(q.device, k=k, v=v)
+    _out(out, "out", torch.bfloat16, (B, Hq, Sq, D), q.device, contiguous=False)
+    _out(lse, "lse", torch.float32, (B, Hq, Sq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -263,6 +321,14 @@ def attn_decode_paged_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: t
     _need(seq_lens, "seq_lens", torch.int32, 1)
     B, Hq, D = q.shape
     P, Hkv, ps, _ = k_pages.shape
+    _shape(k_pages, "k_pages", (P, Hkv, ps, D))
+    _shape(v_pages, "v_pages", k_pages.shape)
+    _shape(block_table, "block_table", (B, block_table.shape[1]))
+    _shape(seq_lens, "seq_lens", (B,))
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens)
+    _out(out, "out", torch.bfloat16, q.shape, q.device)
+    _out(lse, "lse", torch.float32, (B, Hq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -290,6 +356,15 @@ def attn_prefill_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Te
     _need(q_lens, "q_lens", torch.int32, 1)
     B, Hq, max_q, D = q.shape
     P, Hkv, ps, _ = k_pages.shape
+    _shape(k_pages, "k_pages", (P, Hkv, ps, D))
+    _shape(v_pages, "v_pages", k_pages.shape)
+    _shape(block_table, "block_table", (B, block_table.shape[1]))
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(q_lens, "q_lens", (B,))
+    _same_device(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                 seq_lens=seq_lens, q_lens=q_lens)
+    _out(out, "out", torch.bfloat16, q.shape, q.device)
+    _out(lse, "lse", torch.float32, (B, Hq, max_q), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -309,6 +384,10 @@ def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor 
     _need(o_parts, "o_parts", torch.float32, 4)
     _need(lse_parts, "lse_parts", torch.float32, 3)
     S, B, Hq, D = o_parts.shape
+    _shape(lse_parts, "lse_parts", (S, B, Hq))
+    _same_device(o_parts.device, lse_parts=lse_parts)
+    _out(out, "out", torch.bfloat16, (B, Hq, D), o_parts.device)
+    _out(lse, "lse", torch.float32, (B, Hq), o_parts.device)
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=o_parts.device)
     if lse is None and return_lse:

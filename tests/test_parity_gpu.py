@@ -360,6 +360,35 @@ def test_fp8_decode_deterministic(frt):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# ------------------------------------------------ binding argument checks
+def test_binding_rejects_mismatched_tensors(frt):
+    # wrong output shapes, dtypes or table sizes are refused before any kernel
+    # could write or read outside a buffer
+    x = _dev(inputs.dense(1, 4, 2, 64, 64, 64, seed=31))
+    with pytest.raises(ValueError):
+        frt.attn_fwd(x["q"], x["k"], x["v"], out=torch.empty(1, 4, 32, 64, dtype=torch.bfloat16,
+                                                             device="cuda"))
+    with pytest.raises(TypeError):
+        frt.attn_fwd(x["q"], x["k"], x["v"], lse=torch.empty(1, 4, 64, dtype=torch.float16,
+                                                             device="cuda"))
+    with pytest.raises(ValueError):
+        frt.attn_fwd(x["q"], x["k"], x["v"][:, :, :32].contiguous())
+    p = _dev(inputs.paged(2, 8, 2, 128, seq_lens=[40, 50], seed=32))
+    with pytest.raises(ValueError):
+        frt.attn_decode_paged(p["q"], p["k_pages"], p["v_pages"], p["block_table"][:1],
+                              p["seq_lens"])
+    with pytest.raises(ValueError):
+        frt.attn_decode_paged(p["q"], p["k_pages"], p["v_pages"], p["block_table"],
+                              p["seq_lens"][:1])
+    with pytest.raises(ValueError):
+        frt.attn_decode_paged(p["q"], p["k_pages"], p["v_pages"], p["block_table"],
+                              p["seq_lens"], lse=torch.empty(2, 4, device="cuda"))
+    f = _dev(inputs.paged_fp8(2, 8, 2, 128, seq_lens=[40, 50], seed=33))
+    with pytest.raises(ValueError):
+        frt.attn_decode_paged_fp8(f["q"], f["k_pages"], f["v_pages"], f["k_scale"][:1],
+                                  f["v_scale"], f["block_table"], f["seq_lens"])
+
+
 # -------------------------------------------------- exact special cases
 def test_single_visible_key_gives_v_exactly(frt):
     # one key: p = 1 and l = 1, so o is that key's value row, bit for bit
