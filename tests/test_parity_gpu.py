@@ -360,6 +360,24 @@ def test_fp8_decode_deterministic(frt):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_maximum_batch(frt, fp8):
+    # the largest batch the decode plan holds (1024 sequences: 32 per lane of
+    # the prefix scan), ragged lengths including a few empty sequences
+    g = torch.Generator().manual_seed(41)
+    lens = torch.randint(0, 40, (1024,), generator=g).tolist()
+    make = inputs.paged_fp8 if fp8 else inputs.paged
+    x = make(1024, 8, 2, 128, seq_lens=lens, seed=42)
+    if fp8:
+        o, lse = _fp8_case(frt, x, 1 / math.sqrt(128), what="fp8 B=1024")
+    else:
+        o, lse = _paged_case(frt, x, 1 / math.sqrt(128), what="B=1024")
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
+    _no_device_error(frt)
+
+
 # ------------------------------------------------ binding argument checks
 def test_binding_rejects_mismatched_tensors(frt):
     # wrong output shapes, dtypes or table sizes are refused before any kernel
