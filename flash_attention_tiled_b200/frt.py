@@ -119,17 +119,26 @@ def _same_device(device, **tensors):
             raise ValueError(f"{name} is on {t.device}, q on {device}")
 
 
-# Workspaces, one per (device, stream, shape): a call writes every word of
-# the workspace it later reads, so one buffer serves all later calls of the
-# same shape ordered on the same stream.
+# Workspaces, one per (device, stream).  A call writes every word of the
+# workspace it later reads, and each kernel first waits for the one before it
+# in the stream, so one buffer serves every later call on the same stream,
+# whatever its shape.  It grows in powers of two when a call needs more; an
+# outgrown buffer is kept alive (a captured CUDA graph may still use it), so
+# all buffers together hold less than twice the largest need.
 _workspaces: dict = {}
+_retired: list = []
 
 
-def workspace(nbytes: int, device, stream_handle: int, shape_key=()) -> torch.Tensor:
-    key = (torch.device(device).index, stream_handle, nbytes, shape_key)
+def workspace(nbytes: int, device, stream_handle: int) -> torch.Tensor:
+    key = (torch.device(device).index, stream_handle)
     ws = _workspaces.get(key)
-    if ws is None:
-        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+    if ws is None or ws.numel() < nbytes:
+        size = 256
+        while size < nbytes:
+            size *= 2
+        if ws is not None:
+            _retired.append(ws)
+        ws = torch.zeros(size, dtype=torch.uint8, device=device)
         _workspaces[key] = ws
     return ws
 
@@ -160,7 +169,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
                                              stream))
     ws = None
     if need.value > 0:
-        ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, 0))
+        ws = workspace(need.value, q.device, stream.value)
         need = ctypes.c_size_t(ws.numel())
     _check("frt_attn_fwd", _lib.frt_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
                                              Hq, Hkv, Sq, Skv, D, int(causal), scale, _ptr(ws),
@@ -200,7 +209,7 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
     _check("frt_attn_decode_paged", _lib.frt_attn_decode_paged(
         None, None, None, None, block_table.shape[1], None, ps, P, None, None, B, Hq, Hkv, D,
         scale, num_splits, None, ctypes.byref(need), stream))
-    ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, num_splits))
+    ws = workspace(need.value, q.device, stream.value)
     need = ctypes.c_size_t(ws.numel())
     _check("frt_attn_decode_paged", _lib.frt_attn_decode_paged(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), block_table.shape[1],
@@ -248,7 +257,7 @@ def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch
     _check("frt_attn_decode_paged_fp8", _lib.frt_attn_decode_paged_fp8(
         None, None, None, None, None, None, block_table.shape[1], None, ps, P, None, None, B, Hq,
         Hkv, D, scale, num_splits, None, ctypes.byref(need), stream))
-    ws = workspace(need.value, q.device, stream.value, (B, Hq, Hkv, D, num_splits, "fp8"))
+    ws = workspace(need.value, q.device, stream.value)
     need = ctypes.c_size_t(ws.numel())
     _check("frt_attn_decode_paged_fp8", _lib.frt_attn_decode_paged_fp8(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),

@@ -378,6 +378,21 @@ def test_decode_maximum_batch(frt, fp8):
     _no_device_error(frt)
 
 
+def test_decode_workspace_shared_across_shapes(frt):
+    # one workspace per stream serves calls of any shape: a small decode, a
+    # larger one (the buffer grows; the old one is kept), the small one again
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        before = len(frt._retired)
+        for B, lens, seed in ((1, [40], 51), (6, [900, 17, 0, 4000, 33, 1600], 52), (1, [40], 53)):
+            x = inputs.paged(B, 16, 2, 128, seq_lens=lens, seed=seed)
+            _paged_case(frt, x, 1 / math.sqrt(128), what=f"B={B} on a shared workspace")
+        keys = [k for k in frt._workspaces if k[1] == s.cuda_stream]
+        assert len(keys) == 1
+        assert len(frt._retired) >= before + 1
+    _no_device_error(frt)
+
+
 # ------------------------------------------------ binding argument checks
 def test_binding_rejects_mismatched_tensors(frt):
     # wrong output shapes, dtypes or table sizes are refused before any kernel
