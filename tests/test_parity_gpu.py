@@ -382,14 +382,17 @@ def test_decode_workspace_shared_across_shapes(frt):
     # one workspace per stream serves calls of any shape: a small decode, a
     # larger one (the buffer grows; the old one is kept), the small one again
     s = torch.cuda.Stream()
+    g = torch.Generator().manual_seed(50)
+    big = torch.randint(0, 300, (40,), generator=g).tolist()   # 80 segments: a larger need
+    sizes = []
     with torch.cuda.stream(s):
-        before = len(frt._retired)
-        for B, lens, seed in ((1, [40], 51), (6, [900, 17, 0, 4000, 33, 1600], 52), (1, [40], 53)):
+        for B, lens, seed in ((1, [40], 51), (40, big, 52), (1, [40], 53)):
             x = inputs.paged(B, 16, 2, 128, seq_lens=lens, seed=seed)
             _paged_case(frt, x, 1 / math.sqrt(128), what=f"B={B} on a shared workspace")
-        keys = [k for k in frt._workspaces if k[1] == s.cuda_stream]
-        assert len(keys) == 1
-        assert len(frt._retired) >= before + 1
+            keys = [k for k in frt._workspaces if k[1] == s.cuda_stream]
+            assert len(keys) == 1
+            sizes.append(frt._workspaces[keys[0]].numel())
+    assert sizes[1] > sizes[0] and sizes[2] == sizes[1], sizes
     _no_device_error(frt)
 
 
