@@ -159,3 +159,123 @@ def test_fwd_strided_rejects(kw, code):
 
 def test_fwd_strided_empty_is_a_noop():
     assert _strided(B=0) == 0 and _strided(Sq=0) == 0
+
+
+# ------------------------------------------- real calls refused before launch
+# Fake device addresses: these calls are rejected by the argument checks,
+# which run before any CUDA call, so nothing is ever dereferenced.
+A16 = ctypes.c_void_p(1 << 20)         # 16-byte aligned
+ODD = ctypes.c_void_p((1 << 20) + 2)   # 2-byte aligned only
+
+
+def _fwd_call(q=A16, k=A16, v=A16, o=A16, lse=NULL, B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64):
+    need = Z(0)
+    return frt.lib().frt_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, 0, 0.125, NULL,
+                                  ctypes.byref(need), NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(o=NULL), 1),
+    (dict(k=NULL), 1),
+    (dict(q=ODD), 1),
+    (dict(o=ODD), 1),
+    (dict(v=ODD), 1),
+    (dict(lse=ODD), 1),
+    (dict(Sq=1, q=ODD), 1),                     # the decode path checks the same
+    (dict(B=1 << 16, Hq=1 << 8, Hkv=1 << 8, Sq=1 << 8, Skv=1), 2),   # 2^32 query rows
+])
+def test_fwd_real_call_rejects(kw, code):
+    assert _fwd_call(**kw) == code
+
+
+def test_fwd_real_call_with_nothing_to_do():
+    assert _fwd_call(B=0) == 0 and _fwd_call(Sq=0) == 0
+
+
+def _paged_call(q=A16, kp=A16, vp=A16, bt=A16, sl=A16, o=A16, lse=NULL, B=1, Hq=8, Hkv=2,
+                num_pages=4, maxp=2):
+    need = Z(1 << 30)
+    return frt.lib().frt_attn_decode_paged(q, kp, vp, bt, maxp, sl, 16, num_pages, o, lse, B, Hq,
+                                           Hkv, 128, 0.1, 4, A16, ctypes.byref(need), NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kp=NULL), 1),
+    (dict(sl=NULL), 1),
+    (dict(o=NULL), 1),
+    (dict(bt=NULL), 1),
+    (dict(bt=ctypes.c_void_p((1 << 20) + 2)), 1),   # int32 table not 4-byte aligned
+    (dict(sl=ctypes.c_void_p((1 << 20) + 1)), 1),
+    (dict(q=ODD), 1),
+    (dict(lse=ODD), 1),
+    (dict(num_pages=0), 1),
+    (dict(num_pages=1 << 27, Hkv=2), 2),            # 2^32 cache rows
+])
+def test_decode_real_call_rejects(kw, code):
+    assert _paged_call(**kw) == code
+
+
+def _prefill_paged(q=A16, kp=A16, vp=A16, bt=A16, sl=A16, ql=A16, o=A16, lse=NULL, B=1, Hq=4,
+                   Hkv=2, max_q=8, D=128, ps=16, num_pages=4, maxp=2, causal=1, scale=0.1):
+    return frt.lib().frt_attn_prefill_paged(q, kp, vp, bt, maxp, sl, ql, ps, num_pages, o, lse,
+                                            B, Hq, Hkv, max_q, D, causal, scale, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3), 1),
+    (dict(max_q=-1), 1),
+    (dict(causal=2), 1),
+    (dict(scale=0.0), 1),
+    (dict(maxp=-1), 1),
+    (dict(D=80), 2),
+    (dict(ps=32), 2),
+    (dict(num_pages=1 << 27), 2),
+    (dict(q=NULL), 1),
+    (dict(ql=NULL), 1),
+    (dict(bt=NULL), 1),
+    (dict(maxp=0), 1),
+    (dict(num_pages=0), 1),
+    (dict(kp=ODD), 1),
+    (dict(ql=ctypes.c_void_p((1 << 20) + 2)), 1),
+])
+def test_prefill_paged_rejects(kw, code):
+    assert _prefill_paged(**kw) == code
+
+
+def test_prefill_paged_with_nothing_to_do():
+    assert _prefill_paged(B=0) == 0 and _prefill_paged(max_q=0) == 0
+
+
+def test_noalloc_refuses_a_plan_larger_than_its_scratch():
+    # 4000 parts of 16 rows x 128 fp32 partials do not fit the 16 MiB scratch:
+    # refused with FRT_ERR_WORKSPACE before anything runs
+    rc = frt.lib().frt_attn_decode_paged_noalloc(A16, A16, A16, A16, 2, A16, 16, 4, A16, NULL, 1,
+                                                 8, 2, 128, 0.1, 4000, NULL)
+    assert rc == 3
+
+
+def test_noalloc_argument_checks():
+    lib = frt.lib()
+    assert lib.frt_attn_decode_paged_noalloc(A16, A16, A16, A16, 2, A16, 8, 4, A16, NULL, 1, 8, 2,
+                                             128, 0.1, 4, NULL) == 2      # page size 8
+    assert lib.frt_attn_decode_paged_noalloc(NULL, A16, A16, A16, 2, A16, 16, 4, A16, NULL, 1, 8,
+                                             2, 128, 0.1, 4, NULL) == 1   # no q
+    assert lib.frt_attn_decode_paged_noalloc(NULL, NULL, NULL, NULL, 2, NULL, 16, 4, NULL, NULL,
+                                             0, 8, 2, 128, 0.1, 4, NULL) == 0   # empty batch
+
+
+def test_merge_real_call_rejects_misaligned():
+    lib = frt.lib()
+    assert lib.frt_attn_merge_lse(ODD, A16, 2, 1, 4, 64, A16, NULL, NULL) == 1
+    assert lib.frt_attn_merge_lse(A16, A16, 2, 1, 4, 64, ODD, NULL, NULL) == 1
+    assert lib.frt_attn_merge_lse(A16, ctypes.c_void_p((1 << 20) + 1), 2, 1, 4, 64, A16, NULL,
+                                  NULL) == 1
+    assert lib.frt_attn_merge_lse(NULL, A16, 2, 1, 4, 64, A16, NULL, NULL) == 1
+
+
+def test_diagnostic_entries_check_their_arguments():
+    lib = frt.lib()
+    assert lib.frt_read_device_error(None) == 1
+    assert lib.frt_debug_exp2_poly(NULL, NULL, -1, NULL) == 1
+    assert lib.frt_debug_exp2_poly(NULL, NULL, 0, NULL) == 0
+    assert lib.frt_debug_exp2_poly(NULL, NULL, 4, NULL) == 1
