@@ -460,8 +460,8 @@ def run_ours(args, rank, world, local_rank):
     roof["algorithmic_bytes_per_launch"] = round(by / cnt)
     roof["share_of_step"] = round(t_ms / sum(v[0] for v in per_kernel.values()), 3)
 
-    cpu = None
-    if not args.no_cpu_baseline and tuple(names) == Step.ALL:
+    cpu = None   # the oracle on the host cores: rank 0 of a one-GPU run only
+    if not args.no_cpu_baseline and world == 1 and tuple(names) == Step.ALL:
         cpu = cpu_baseline(st)
     line = {
         "metric": METRIC,
