@@ -490,7 +490,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": sum(Step.LAUNCHES[n] for n in names) * args.steps,
+        "gpu_launches": sum(Step.LAUNCHES[n] for n in names) * args.steps * world,   # all ranks
         "clocks": sampler.summary(),
     }
     return line
