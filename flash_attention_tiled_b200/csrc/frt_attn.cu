@@ -432,6 +432,21 @@ __global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
   }
 }
 
+// One thread waits on an mbarrier that nothing arrives at, with the bounded
+// wait every kernel of the library uses: it must give up after its limit,
+// raise the time-out bit of the device error word and return.  *returned
+// becomes 2 when the wait gave up, 1 if it (wrongly) completed.
+__global__ void wait_timeout_selftest_kernel(int* returned) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    *returned = mbar_wait(&bar, 0u, &abort_flag) ? 1 : 2;
+  }
+}
+
 __global__ void fp8_decode_selftest_kernel(const uint8_t* codes, float* y, int n) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (i < n) {
@@ -675,6 +690,12 @@ frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t str
   if (n == 0) return FRT_OK;
   const int pairs = (n + 1) / 2;
   exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+frt_status frt_debug_wait_timeout(int* returned, cudaStream_t stream) {
+  if (returned == nullptr || !aligned16(returned)) return FRT_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(returned);
   return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
 }
 

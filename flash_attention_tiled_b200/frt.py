@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
            "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8", "frt_attn_fwd_strided",
            "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
-           "frt_debug_fp8_decode", "frt_version")
+           "frt_debug_fp8_decode", "frt_debug_wait_timeout", "frt_version")
 
 STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
           3: "FRT_ERR_WORKSPACE", 4: "FRT_ERR_CUDA"}
@@ -50,6 +50,7 @@ def _load() -> ctypes.CDLL:
     lib.frt_attn_decode_paged_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I,
                                               P, Z, P]
     lib.frt_debug_fp8_decode.argtypes = [P, P, I, P]
+    lib.frt_debug_wait_timeout.argtypes = [P, P]
     lib.frt_attn_fwd_strided.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, P, P]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = ctypes.c_int

@@ -301,6 +301,16 @@ FRT_API frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_par
 FRT_API frt_status frt_read_device_error(unsigned* flags);
 
 /*
+ * frt_debug_wait_timeout -- failure-detection self-test: one thread waits on
+ * an mbarrier that nothing arrives at, through the same bounded wait every
+ * kernel uses.  After the wait limit (2 s) it gives up, sets bit 0 of the
+ * device error word (see frt_read_device_error) and writes 2 to *returned
+ * (1 would mean the wait completed, which it must not).  The context stays
+ * usable.  returned: one device int32, 16-byte aligned.
+ */
+FRT_API frt_status frt_debug_wait_timeout(int* returned, cudaStream_t stream);
+
+/*
  * frt_debug_exp2_poly -- diagnostic: y[i] = the library's FMA-pipe 2^x for
  * x[i] (device arrays of n floats; inputs below -125 are clamped there).
  * The prefill kernel's softmax can compute part of its exponentials this way

@@ -6,6 +6,7 @@ page, which slot) bit-exact.  The five named workloads run at full size;
 where the oracle would take too long (the 4k prefill) it checks sampled rows,
 computed one by one, of the very launch the benchmark times.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -393,6 +394,28 @@ def test_decode_workspace_shared_across_shapes(frt):
             assert len(keys) == 1
             sizes.append(frt._workspaces[keys[0]].numel())
     assert sizes[1] > sizes[0] and sizes[2] == sizes[1], sizes
+    _no_device_error(frt)
+
+
+def test_a_wait_nothing_ends_times_out_and_the_context_survives(frt):
+    # failure detection without a fault: a wait on a barrier that nothing
+    # arrives at gives up after its limit and reports it on the host
+    import time
+    lib = frt.lib()
+    flags = ctypes.c_uint(0)
+    torch.cuda.synchronize()
+    assert lib.frt_read_device_error(ctypes.byref(flags)) == 0        # clear
+    r = torch.zeros(4, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    assert lib.frt_debug_wait_timeout(ctypes.c_void_p(r.data_ptr()), None) == 0
+    torch.cuda.synchronize()
+    took = time.time() - t0
+    assert r[0].item() == 2
+    assert 1.0 < took < 60.0, took
+    assert lib.frt_read_device_error(ctypes.byref(flags)) == 0 and (flags.value & 1)
+    # the context still runs real work
+    x = inputs.paged(1, 8, 2, 128, seq_lens=[100], seed=61)
+    _paged_case(frt, x, 1 / math.sqrt(128), what="after a timed-out wait")
     _no_device_error(frt)
 
 
