@@ -478,6 +478,8 @@ frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void*
   if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
   if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
   if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  // the kernel's page prefix over the batch is 32-bit
+  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
   if (q != nullptr && B > 0) {
     if (k_pages == nullptr || v_pages == nullptr || o == nullptr ||
         seq_lens == nullptr || (block_table == nullptr && max_pages_per_seq > 0))
@@ -508,6 +510,7 @@ frt_status frt_attn_decode_paged_fp8(const void* q, const void* k_pages, const v
   if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
   if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
   if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
   if (q != nullptr && B > 0) {
     if (k_pages == nullptr || v_pages == nullptr || o == nullptr || k_scale == nullptr ||
         v_scale == nullptr || seq_lens == nullptr ||
@@ -604,7 +607,8 @@ frt_status frt_attn_prefill_paged(const void* q, const void* k_pages, const void
   if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
   if (page_size != 16) return FRT_ERR_UNSUPPORTED;
   if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31) ||
-      (uint64_t)B * Hq * max_q >= (1ull << 31))
+      (uint64_t)B * Hq * max_q >= (1ull << 31) ||
+      (uint64_t)max_pages_per_seq * page_size >= (1ull << 31))   // 32-bit length bound
     return FRT_ERR_UNSUPPORTED;
   if (B == 0 || max_q == 0) return FRT_OK;
   if (q == nullptr || o == nullptr || k_pages == nullptr || v_pages == nullptr ||

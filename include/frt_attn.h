@@ -135,8 +135,8 @@ FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, voi
  * bounds), never out-of-bounds memory.  Tail slots of the last page of a
  * sequence may hold anything, NaN included: they never reach o.
  *
- * Size limit (not checked in this version): the pages of all sequences
- * together, B * max_pages_per_seq, must stay below 2^31, since the kernel
+ * Size limit: the pages of all sequences together, B * max_pages_per_seq,
+ * must stay below 2^31 (FRT_ERR_UNSUPPORTED otherwise), since the kernel
  * counts pages in 32 bits.  Sequences may share physical pages, so this
  * limits the block table, not the cache.  Reaching it takes a block table
  * of 8 GB or more.
@@ -173,8 +173,9 @@ FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, con
  * through the block table.  Needs no workspace.  Tail slots of a sequence's
  * last page may hold anything, NaN included.
  *
- * Size limit (not checked in this version): max_pages_per_seq * 16 must stay
- * below 2^31, since a sequence's length bound is computed in 32 bits.
+ * Size limit: max_pages_per_seq * 16 must stay below 2^31
+ * (FRT_ERR_UNSUPPORTED otherwise), since a sequence's length bound is
+ * computed in 32 bits.
  */
 FRT_API frt_status frt_attn_prefill_paged(const void* q, const void* k_pages,
                                           const void* v_pages, const int32_t* block_table,

@@ -279,3 +279,14 @@ def test_diagnostic_entries_check_their_arguments():
     assert lib.frt_debug_exp2_poly(NULL, NULL, -1, NULL) == 1
     assert lib.frt_debug_exp2_poly(NULL, NULL, 0, NULL) == 0
     assert lib.frt_debug_exp2_poly(NULL, NULL, 4, NULL) == 1
+
+
+def test_page_count_limits_are_checked():
+    # B * max_pages_per_seq >= 2^31 (paged decode, bf16 and FP8) and
+    # max_pages_per_seq * 16 >= 2^31 (chunked prefill) are refused
+    assert _paged_call(B=1024, maxp=1 << 21) == 2
+    need = Z(0)
+    assert frt.lib().frt_attn_decode_paged_fp8(NULL, NULL, NULL, NULL, NULL, NULL, 1 << 21, NULL, 16,
+                                               10, NULL, NULL, 1024, 8, 2, 128, 0.1, 4, NULL,
+                                               ctypes.byref(need), NULL) == 2
+    assert _prefill_paged(maxp=1 << 27) == 2
