@@ -1,13 +1,15 @@
 """Benchmark of the fused-attention hot path on B200.
 
 One step = one pass of every operation on the path over its own seeded,
-HBM-resident synthetic input:
+HBM-resident synthetic input (the five workloads):
+  tiny      tiny causal self-attention         B1 Hq2 Hkv2 S128 D64     (frt_attn_fwd)
   prefill   Llama-3-8B-shaped causal prefill   B1 Hq32 Hkv8 S4096 D128  (frt_attn_fwd)
   paged     paged GQA decode                   B4 Hq64 Hkv8 D128 ps16, lens U[1024,32768]
                                                (frt_attn_decode_paged: streaming kernel,
                                                then the dependent LSE merge kernel)
   long      long-context split-KV decode       B1 Hq32 Hkv4 Skv262144 D128 ps16
-  contig    single-token GQA decode            B1 Hq32 Hkv8 Skv4096 D128 (frt_attn_fwd, Sq=1)
+  contig    single-token GQA decode            B1 Hq32 Hkv8 Skv4096 D128 (frt_attn_fwd, Sq=1:
+                                               one launch, clusters merge in shared memory)
 Each step's working set (~0.9 GB) exceeds the 126 MB L2, and every call's
 inputs are evicted by the calls before it, so no call starts L2-warm.
 
@@ -19,8 +21,9 @@ attention, the prefill through strided views), timed the same way.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
---impl reference times the CPU oracle (fp64, OpenMP) on the host cores on a
-bounded sample of the same step (rank 0 only).
+--impl reference times the CPU oracle (fp64, OpenMP) on the host cores: each
+step is one full pass of the oracle over the same five workloads (rank 0
+only).
 """
 from __future__ import annotations
 
@@ -43,10 +46,13 @@ from flash_attention_tiled_b200 import inputs  # noqa: E402
 
 METRIC = ("attn prefill TFLOP/s & decode KV GB/s vs B200 roofline; "
           "µs/call at batch 1")
-WORKLOAD = ("llama3-8b causal prefill 4k (B1 Hq32 Hkv8 D128) + paged GQA decode "
-            "(B4 Hq64 Hkv8 D128 ps16 lens U[1024,32768]) + 256k split-KV decode "
-            "(B1 Hq32 Hkv4 D128 ps16) + 4k GQA decode (B1 Hq32 Hkv8 D128)")
+WORKLOAD = ("tiny causal (B1 H2 S128 D64) + llama3-8b causal prefill 4k (B1 Hq32 Hkv8 D128) "
+            "+ paged GQA decode (B4 Hq64 Hkv8 D128 ps16 lens U[1024,32768]) + 256k split-KV "
+            "decode (B1 Hq32 Hkv4 D128 ps16) + 4k GQA decode (B1 Hq32 Hkv8 D128)")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREROLL_S = 1.5          # untimed step replays under the clock sampler before the timed steps
+REF_STEP_S_EST = 5.0     # one full oracle step on 16 host cores (seconds, for run planning)
+REF_BUDGET_S = 240.0     # the reference arm's planned length
 
 
 def source_sha() -> str:
@@ -183,15 +189,16 @@ class ClockSampler:
 
 # -------------------------------------------------------------- our arm
 class Step:
-    """The four calls of one step, with inputs resident on the device."""
+    """The five calls of one step, with inputs resident on the device."""
 
-    ALL = ("prefill", "paged", "long", "contig")
+    ALL = ("tiny", "prefill", "paged", "long", "contig")
     # the paged workloads with their cache stored as e4m3 (not part of the
     # configured step; --calls may name them, e.g. for a profile)
     FP8 = ("paged_fp8", "long_fp8")
     # kernels each call launches: prefill_kernel; decode_splitkv_kernel then
-    # decode_merge_kernel
-    LAUNCHES = {"prefill": 1, "paged": 2, "long": 2, "contig": 2, "paged_fp8": 2, "long_fp8": 2}
+    # decode_merge_kernel (paged); the cluster-mode decode kernel alone (contig)
+    LAUNCHES = {"tiny": 1, "prefill": 1, "paged": 2, "long": 2, "contig": 1, "paged_fp8": 2,
+                "long_fp8": 2}
 
     def __init__(self, device, names=ALL):
         from flash_attention_tiled_b200 import frt
@@ -199,12 +206,13 @@ class Step:
         self.dev = device
         self.NAMES = tuple(names)
         W = inputs.WORKLOADS
+        self.w_tn = W["tiny_causal"]
         self.w_pf = W["llama3_8b_prefill_4k"]
         self.w_pg = W["paged_gqa_decode_b4"]
         self.w_lg = W["long_splitkv_decode_256k"]
         self.w_ct = W["gqa_decode_4k"]
-        wl = {"prefill": self.w_pf, "paged": self.w_pg, "long": self.w_lg, "contig": self.w_ct,
-              "paged_fp8": self.w_pg, "long_fp8": self.w_lg}
+        wl = {"tiny": self.w_tn, "prefill": self.w_pf, "paged": self.w_pg, "long": self.w_lg,
+              "contig": self.w_ct, "paged_fp8": self.w_pg, "long_fp8": self.w_lg}
 
         def make(n):
             w = wl[n]
@@ -223,7 +231,8 @@ class Step:
         self.tokens = {n: int(self.host[n]["seq_lens"].sum()) for n in self.NAMES
                        if n in Step.FP8}
         # outputs, allocated once
-        shapes = {"prefill": (self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq),
+        shapes = {"tiny": (self.w_tn.B, self.w_tn.Hq, self.w_tn.Sq),
+                  "prefill": (self.w_pf.B, self.w_pf.Hq, self.w_pf.Sq),
                   "paged": (self.w_pg.B, self.w_pg.Hq), "long": (self.w_lg.B, self.w_lg.Hq),
                   "contig": (self.w_ct.B, self.w_ct.Hq, 1),
                   "paged_fp8": (self.w_pg.B, self.w_pg.Hq), "long_fp8": (self.w_lg.B, self.w_lg.Hq)}
@@ -234,7 +243,9 @@ class Step:
         d = self.d[name] if d is None else d
         o, l = self.out[name] if out is None else out
         f = self.frt
-        if name == "prefill":
+        if name == "tiny":
+            f.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=self.w_tn.scale, out=o, lse=l)
+        elif name == "prefill":
             f.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=self.w_pf.scale, out=o, lse=l)
         elif name == "contig":
             f.attn_fwd(d["q"], d["k"], d["v"], causal=False, scale=self.w_ct.scale, out=o, lse=l)
@@ -251,7 +262,9 @@ class Step:
         """Algorithmic (flops, bytes) of each call."""
         out = {}
         for n in self.NAMES:
-            if n == "prefill":
+            if n == "tiny":
+                out[n] = (prefill_flops(self.w_tn), prefill_bytes(self.w_tn))
+            elif n == "prefill":
                 out[n] = (prefill_flops(self.w_pf), prefill_bytes(self.w_pf))
             elif n == "paged":
                 out[n] = (decode_flops(self.w_pg.Hq, 128, self.tokens_pg),
@@ -346,8 +359,20 @@ def run_ours(args, rank, world, local_rank):
 
     sync_ranks(world)
     torch.cuda.synchronize(device)
+    # The clock sampler (nvidia-smi, one sample per 100 ms) runs through a
+    # pre-roll of untimed step replays lasting PREROLL_S seconds and then
+    # through the K timed steps, which alone are too short to be sampled.
     sampler = ClockSampler(device.index if device.index is not None else 0)
+    preroll = 0
     with sampler, torch.cuda.stream(stream):
+        t_end = time.perf_counter() + PREROLL_S
+        while time.perf_counter() < t_end:
+            for _ in range(50):
+                g_step.replay()
+            preroll += 50
+            torch.cuda.synchronize(device)
+        sync_ranks(world)
+        torch.cuda.synchronize(device)
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         start.record(stream)
@@ -375,6 +400,20 @@ def run_ours(args, rank, world, local_rank):
 
     t_flush = graph_ms(g_flush)
     per_call_ms = {n: max(graph_ms(g_call[n]) - t_flush, 1e-6) / R for n in names}
+    # the tiny call once more as a host program makes it: 200 eager calls
+    # through the binding back to back (host marshalling and launch included)
+    eager_us = None
+    if "tiny" in names:
+        with torch.cuda.stream(stream):
+            for _ in range(20):
+                st.call("tiny")
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(200):
+                st.call("tiny")
+            b.record(stream)
+            torch.cuda.synchronize(device)
+        eager_us = a.elapsed_time(b) / 200 * 1e3
     # the contiguous decode once more with its inputs left in L2: R calls back
     # to back, no flush (reported beside the flushed figure, labelled L2-hot)
     hot_ms = None
@@ -415,12 +454,15 @@ def run_ours(args, rank, world, local_rank):
         us = per_call_ms[n] * 1e3
         rec = {"us": round(us, 2), "tflops": round(fl / us * 1e-6, 1),
                "gbs": round(by / us * 1e-3, 1), "flop": fl, "bytes": by}
-        if n == "prefill":
-            rec["bound"] = "tensor"
+        if n in ("prefill", "tiny"):
+            rec["bound"] = "tensor" if n == "prefill" else "latency"
             rec["frac"] = round(rec["tflops"] / peaks["bf16_tflops"], 4)
         else:
             rec["bound"] = "hbm"
             rec["frac"] = round(rec["gbs"] / peaks["hbm_gbs"], 4)
+        if n == "tiny" and eager_us is not None:
+            rec["eager"] = {"us": round(eager_us, 2),
+                            "note": "200 eager calls back to back through the Python binding"}
         if n == "contig" and hot_ms is not None:
             rec["l2_hot"] = {"us": round(hot_ms * 1e3, 2),
                              "gbs": round(by / (hot_ms * 1e3) * 1e-3, 1),
@@ -430,8 +472,10 @@ def run_ours(args, rank, world, local_rank):
     # decode kernel serves three calls, the prefill kernel one.  A decode
     # call's time also holds its small merge kernel (timed together, so the
     # streaming kernel's fraction is if anything understated).
-    kernel_of = {"prefill": "prefill_kernel<128>", "paged": "decode_splitkv_kernel<128>",
-                 "long": "decode_splitkv_kernel<128>", "contig": "decode_splitkv_kernel<128>",
+    kernel_of = {"tiny": "prefill_kernel<64>", "prefill": "prefill_kernel<128>",
+                 "paged": "decode_splitkv_kernel<128>",
+                 "long": "decode_splitkv_kernel<128>",
+                 "contig": "decode_splitkv_kernel<128> (cluster mode)",
                  "paged_fp8": "decode_splitkv_kernel<128> (e4m3 cache)",
                  "long_fp8": "decode_splitkv_kernel<128> (e4m3 cache)"}
     per_kernel = {}
@@ -491,7 +535,9 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": sum(Step.LAUNCHES[n] for n in names) * args.steps * world,   # all ranks
-        "clocks": sampler.summary(),
+        "clocks": dict(sampler.summary(), window=(
+            f"{PREROLL_S:.0f} s of untimed step replays ({preroll} steps) immediately before "
+            f"the timed region, and the timed region")),
     }
     return line
 
@@ -626,64 +672,54 @@ def run_e2e(st: Step, args, device):
 
 
 # ------------------------------------------------------------- oracle arm
-def cpu_sample_plan():
-    """Bounded oracle sample of one step and the factor scaling it to a full step:
-    prefill on 8 of 32 query heads (full causal rows), paged decode on 16 of
-    256 rows, long decode on 4 of 32 heads, contiguous decode on all 32 heads."""
-    return {"prefill_heads": 8, "paged_rows": 16, "long_heads": 4}
-
-
 def cpu_baseline(st: Step | None, host=None):
+    """One full step of the oracle on the host cores: every call of the step
+    at its full size (the fp64 oracle as it stands, OpenMP over its
+    (sequence, head) rows), timed by wall clock."""
     import oracle
-    plan = cpu_sample_plan()
     W = inputs.WORKLOADS
     if host is None:
         host = st.host
-    t_total = 0.0
+    legs = {}
     t0 = time.perf_counter()
-    # prefill: the first `prefill_heads` query heads with their KV heads
-    w = W["llama3_8b_prefill_4k"]
-    x = host["prefill"]
-    hq = plan["prefill_heads"]
-    g = w.Hq // w.Hkv
-    hkv = (hq + g - 1) // g
-    ts = time.perf_counter()
-    oracle.attn_fwd(x["q"][:, :hq].contiguous(), x["k"][:, :hkv].contiguous(),
-                    x["v"][:, :hkv].contiguous(), True, w.scale)
-    t_total += (time.perf_counter() - ts) * (w.Hq / hq)
-    # paged decode: a mask of rows
-    for name, key, rows_key in (("paged_gqa_decode_b4", "paged", "paged_rows"),
-                                ("long_splitkv_decode_256k", "long", "long_heads")):
-        w = W[name]
-        x = host[key]
-        n_rows = plan[rows_key]
-        mask = np.zeros((w.B, w.Hq), dtype=bool)
-        mask.reshape(-1)[:n_rows] = True
+    for key, name in (("tiny", "tiny_causal"), ("prefill", "llama3_8b_prefill_4k"),
+                      ("contig", "gqa_decode_4k")):
+        w, x = W[name], host[key]
+        ts = time.perf_counter()
+        oracle.attn_fwd(x["q"], x["k"], x["v"], w.causal, w.scale)
+        legs[key] = time.perf_counter() - ts
+    for key, name in (("paged", "paged_gqa_decode_b4"), ("long", "long_splitkv_decode_256k")):
+        w, x = W[name], host[key]
         ts = time.perf_counter()
         oracle.attn_decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"],
-                                 x["seq_lens"], w.scale, heads_mask=mask)
-        t_total += (time.perf_counter() - ts) * (w.B * w.Hq / n_rows)
-    w = W["gqa_decode_4k"]
-    x = host["contig"]
-    ts = time.perf_counter()
-    oracle.attn_fwd(x["q"], x["k"], x["v"], False, w.scale)
-    t_total += time.perf_counter() - ts
-    wall = time.perf_counter() - t0
-    return {"value": round(1.0 / t_total, 6), "unit": "step/s", "cores": oracle.threads(),
+                                 x["seq_lens"], w.scale)
+        legs[key] = time.perf_counter() - ts
+    total = time.perf_counter() - t0
+    return {"value": round(1.0 / total, 6), "unit": "step/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": (f"one step sampled: prefill {plan['prefill_heads']}/32 heads, paged "
-                       f"decode {plan['paged_rows']}/256 rows, long decode "
-                       f"{plan['long_heads']}/32 heads, contiguous decode all 32 heads; "
-                       f"each leg's time scaled by its sampled fraction "
-                       f"({wall:.1f} s of CPU wall time)"),
-            "s_per_step": round(t_total, 3)}
+            "sample": "one full step: all five calls at full size, nothing extrapolated",
+            "s_per_step": round(total, 3),
+            "s_per_call": {k: round(v, 4) for k, v in legs.items()}}
+
+
+def reference_plan(steps: int, warmup: int):
+    """(timed, untimed) oracle steps of the reference arm: the GPU arm's K and W
+    when they fit the planned length, else as many timed steps as fit."""
+    budget = max(1, int(REF_BUDGET_S // REF_STEP_S_EST))
+    timed = max(1, min(steps, budget))
+    return timed, max(0, min(warmup, budget - timed))
+
+
+def reference_host_inputs():
+    return {"tiny": inputs.make("tiny_causal"), "prefill": inputs.make("llama3_8b_prefill_4k"),
+            "paged": inputs.make("paged_gqa_decode_b4"),
+            "long": inputs.make("long_splitkv_decode_256k"), "contig": inputs.make("gqa_decode_4k")}
 
 
 def run_reference(args, rank):
     if rank != 0:
         return None
-    host = {"prefill": inputs.make("llama3_8b_prefill_4k"), "paged": inputs.make("paged_gqa_decode_b4"),
-            "long": inputs.make("long_splitkv_decode_256k"), "contig": inputs.make("gqa_decode_4k")}
+    host = reference_host_inputs()
     for _ in range(args.warmup_ref):
         cpu_baseline(None, host=host)
     vals = [cpu_baseline(None, host=host) for _ in range(args.steps_ref)]
@@ -691,6 +727,7 @@ def run_reference(args, rank):
     cb = vals[-1]
     value = round(1.0 / s_per_step, 6)
     cb["value"] = value
+    cb["s_per_step"] = round(s_per_step, 3)
     return {
         "impl": "reference",
         "metric": METRIC, "value": value, "unit": "step/s", "n_gpus": 1,
@@ -699,7 +736,8 @@ def run_reference(args, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, shuffled page tables)",
         "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
-                   "parallelism": "host cores (OpenMP)"},
+                   "parallelism": "host cores (OpenMP)",
+                   "timing": "wall clock around each full oracle step"},
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "step/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -731,9 +769,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        # each oracle step is a bounded sample of ~10 s; keep the run to minutes
-        args.steps_ref = max(1, min(args.steps, 3))
-        args.warmup_ref = 0
+        # every step is one full oracle pass (~5 s on 16 host cores): K timed
+        # steps after W untimed ones, as many as the GPU arm runs, unless that
+        # would take more than ~4 minutes (the default K of 2000 would)
+        args.steps_ref, args.warmup_ref = reference_plan(args.steps, args.warmup)
         line = run_reference(args, rank)
         if line is not None:
             print(json.dumps(line), flush=True)

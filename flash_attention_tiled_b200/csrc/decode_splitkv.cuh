@@ -33,6 +33,14 @@
 // of its group.  Scores live in the exp2 domain (scale * log2(e) folded in).
 // At the end of a piece the warps' states are combined in registers (through
 // shared memory) and written by one warp.
+//
+// Cluster mode (kCluster, contiguous cache only): no workspace and no second
+// kernel.  Each segment is owned by one thread-block cluster of C <= 16 CTAs;
+// CTA r of the cluster streams pages [r*n/C, (r+1)*n/C) of the segment's n
+// pages, leaves its state (unnormalised output, running max and both sums)
+// in its own shared memory, and after a cluster barrier the cluster's
+// threads merge the C states by log-sum-exp, reading the other CTAs' shared
+// memory directly (distributed shared memory), and write the final rows.
 #pragma once
 
 #include "frt_device.cuh"
@@ -69,6 +77,9 @@ struct DecodeParams {
   const int32_t* block_table;    // paged: [B, max_pages]; contiguous: nullptr
   const int32_t* seq_lens;       // paged: [B] (device); contiguous: nullptr
   int max_pages;                 // paged: block-table row length
+  int num_pages;                 // paged: physical pages; entries outside [0, num_pages)
+                                 // are read from row `bad_row` (past the end: zeros)
+  int bad_row;                   // rows of the [rows, D] view of the cache (< 2^31)
   int contig_len;                // contiguous: keys per sequence (Skv)
   int B, Hq, Hkv, g, hgroups;    // g = Hq / Hkv, hgroups = ceil(g / 16)
   int parts;                     // CTAs of the streaming kernel's grid
@@ -99,6 +110,12 @@ struct DecodeSmem {
   // 2 heads of each head tile)
   static constexpr int kFragFloats = (D / 16) * kHT * 4 + 6 * kHT;
   static constexpr int kScratchFloats = (Cfg::kWarps / 2) * kFragFloats * 32;
+  // cluster mode: a CTA's final state reuses the scratch area: unnormalised
+  // o of up to 8 * kHT heads, then per head {running max, sum of the rounded
+  // weights, exact sum, unused} (one 16-byte load)
+  static constexpr int kXchO = 0;
+  static constexpr int kXchS = kHT * 8 * D;
+  static_assert(kXchS + kHT * 8 * 4 <= kScratchFloats, "cluster exchange fits in the scratch area");
   static constexpr int kScratchOff = kRingBytes;
   static constexpr int kPrefixOff = kScratchOff + kScratchFloats * 4;
   static constexpr int kBarOff = kPrefixOff + ((kDecMaxBatch + 1) * 4 + 15) / 16 * 16;
@@ -153,10 +170,13 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int 
 // loaded by ldmatrix as byte quadruples, so the MMA's k index walks d in the
 // order (4c, 4c+1 | 4c+2, 4c+3) per 16-d step, and Q's fragments follow the
 // same order; V^T's rows come out as the even and odd d of each pair.
-template <int D, int kHT, bool kFp8>
+// kCluster: cluster mode (see the top of this file): contiguous bf16 cache,
+// launched with a cluster of C CTAs per segment; nothing goes to a workspace.
+template <int D, int kHT, bool kFp8, bool kCluster = false>
 __global__ void __launch_bounds__(DecodeCfg<kFp8, kHT>::kThreads, kDecCtasPerSm)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  static_assert(!(kCluster && kFp8), "cluster mode reads a bf16 cache");
   using L = DecodeSmem<D, kFp8, kHT>;
   constexpr int kDecWarps = DecodeCfg<kFp8, kHT>::kWarps;            // consumer warps
   constexpr int kDecStagePages = DecodeCfg<kFp8, kHT>::kStagePages;
@@ -184,9 +204,10 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   griddep_wait();
   griddep_launch_dependents();
 
-  // ---- per-sequence page prefix (warp 0: chunked scan), barriers
+  // ---- per-sequence page prefix (warp 0: chunked scan; not needed in
+  // cluster mode, where every sequence has contig_len keys), barriers
   if (warp == 0) {
-    const int per = (p.B + 31) / 32;
+    const int per = kCluster ? 0 : (p.B + 31) / 32;
     const int b0 = lane * per;
     int local = 0;
     for (int i = 0; i < per; ++i)
@@ -202,7 +223,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         prefix[b0 + i] = run;
         run += dec_pages_of(p, b0 + i);
       }
-    if (lane == 31) prefix[p.B] = incl;
+    if (!kCluster && lane == 31) prefix[p.B] = incl;
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
         mbar_init(&full_bar[s], 1);
@@ -216,12 +237,17 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
   }
   __syncthreads();
 
-  const long long T = (long long)prefix[p.B] * nseg_b;   // total units
-  const int C = (int)min((long long)gridDim.x, T);       // CTAs with a non-empty share
+  // unit line (split mode): T units over the C CTAs with a non-empty share
+  const long long T = kCluster ? 0 : (long long)prefix[p.B] * nseg_b;
+  const int C = kCluster ? 0 : (int)min((long long)gridDim.x, T);
   const int c = blockIdx.x;
+  // cluster mode: segment of this cluster, and this CTA's rank among its CTAs
+  const int cl_size = kCluster ? (int)cluster_nctarank() : 1;
+  const int cl_rank = kCluster ? (int)cluster_ctarank() : 0;
+  const int cl_seg = c / cl_size;
 
   // ---- sequences with no key: o = 0, lse = -inf (spread over the grid)
-  for (int b = c; b < p.B; b += gridDim.x) {
+  for (int b = c; !kCluster && b < p.B; b += gridDim.x) {
     if (prefix[b + 1] != prefix[b]) continue;
     for (int i = threadIdx.x; i < p.Hq * D; i += blockDim.x)
       p.o[(size_t)b * p.Hq * D + i] = __float2bfloat16(0.f);
@@ -229,10 +255,10 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
       for (int i = threadIdx.x; i < p.Hq; i += blockDim.x) p.lse[(size_t)b * p.Hq + i] = -INFINITY;
     for (int i = threadIdx.x; i < nseg_b; i += blockDim.x) p.ws_seg[(size_t)b * nseg_b + i] = make_int2(-1, -1);
   }
-  if (c >= C) return;
+  if (!kCluster && c >= C) return;
 
-  const long long u_begin = (long long)c * T / C;
-  const long long u_end = (long long)(c + 1) * T / C;
+  const long long u_begin = kCluster ? 0 : (long long)c * T / C;
+  const long long u_end = kCluster ? 0 : (long long)(c + 1) * T / C;
 
   // Walk of this CTA's pieces, identical in every warp.  Returns false when
   // the share is exhausted.  (b, seg_in_b) identify the segment, pages
@@ -242,6 +268,18 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     long long seg_u0;
   };
   auto first_piece = [&](Piece& pc) {
+    if constexpr (kCluster) {
+      // the cluster's segment; this CTA's equal share of its pages (may be
+      // empty when the segment has fewer pages than the cluster has CTAs)
+      const int npg = (p.contig_len + kDecPage - 1) / kDecPage;
+      pc.b = cl_seg / nseg_b;
+      pc.seg_in_b = cl_seg % nseg_b;
+      pc.npg = npg;
+      pc.seg_u0 = 0;
+      pc.pg0 = (int)((long long)cl_rank * npg / cl_size);
+      pc.pg1 = (int)((long long)(cl_rank + 1) * npg / cl_size);
+      return;
+    }
     // largest b with prefix[b] * nseg_b <= u_begin and a non-empty sequence
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
@@ -261,6 +299,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     pc.pg1 = (int)((seg_end < u_end ? seg_end : u_end) - pc.seg_u0);
   };
   auto next_piece = [&](Piece& pc) -> bool {
+    if (kCluster) return false;   // one piece per CTA
     long long u = pc.seg_u0 + pc.pg1;
     if (u >= u_end) return false;
     int b = pc.b, s = pc.seg_in_b + 1;
@@ -295,10 +334,19 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (lane < n) {
           const int page = pb + lane;
           if (p.block_table != nullptr) {
+            // An entry outside [0, num_pages) is never used as an address:
+            // the copy starts past the cache's last row, so the page reads as
+            // zeros, and the error word records it.  Valid rows are below
+            // num_pages * Hkv * 16 < 2^31 (checked by the host).
             const int phys = p.block_table[(size_t)pc.b * p.max_pages + page];
-            row = (phys * p.Hkv + kvh) * kDecPage;
+            if ((unsigned)phys < (unsigned)p.num_pages) {
+              row = (int)(((long long)phys * p.Hkv + kvh) * kDecPage);
+            } else {
+              row = p.bad_row;
+              raise_error(kErrBadPage);
+            }
           } else {
-            row = ((pc.b * p.Hkv + kvh) * p.contig_len) + page * kDecPage;
+            row = (int)(((long long)pc.b * p.Hkv + kvh) * p.contig_len + (long long)page * kDecPage);
           }
         }
         ok = mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag);
@@ -323,8 +371,7 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // here before the CTA can finish.  After an abort they may not, so give
     // copies still in flight time to land before this warp leaves.
     if (!ok) __nanosleep(100000);
-    return;
-  }
+  } else {
 
   // ====================================================== consumers (MMA)
   // S^T = K.Q^T with a page's 16 tokens as the MMA M dimension and the
@@ -662,11 +709,36 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
       asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));
     }
 
-    // ---- warp 0 writes the piece: the final rows, or one partial
+    // ---- warp 0 writes the piece: the final rows, or one partial (cluster
+    // mode: this CTA's state, into its own shared memory)
     const int seg = pc.b * nseg_b + pc.seg_in_b;
-    const bool whole = (pc.pg0 == 0) && (pc.pg1 == pc.npg);
+    const bool whole = kCluster ? (cl_size == 1) : (pc.pg0 == 0) && (pc.pg1 == pc.npg);
     const int slot = c + seg;
-    if (cw == 0) {
+    if (kCluster && !whole) {
+      if (cw == 0) {
+#pragma unroll
+        for (int ht = 0; ht < kHT; ++ht)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float ls = l_run[ht][hh], le = le_run[ht][hh];
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+              ls += __shfl_xor_sync(0xffffffffu, ls, off);
+              le += __shfl_xor_sync(0xffffffffu, le, off);
+            }
+            const int r = ht * 8 + 2 * qc + hh;   // head within the segment
+            float* xo = scratch + L::kXchO + r * D;
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+              xo[mt * 16 + r8] = acc[mt][ht][hh];
+              xo[mt * 16 + 8 + r8] = acc[mt][ht][2 + hh];
+            }
+            if (r8 == 0)
+              *reinterpret_cast<float4*>(scratch + L::kXchS + 4 * r) =
+                  make_float4(m_run[ht][hh], ls, le, 0.f);
+          }
+      }
+    } else if (cw == 0) {
 #pragma unroll
       for (int ht = 0; ht < kHT; ++ht)
 #pragma unroll
@@ -714,11 +786,76 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
         }
       // the owner of the segment's first page records where its pieces are
-      if (pc.pg0 == 0 && lane == 0)
+      // (cluster mode has no workspace: a one-CTA cluster writes its rows whole)
+      if (!kCluster && pc.pg0 == 0 && lane == 0)
         p.ws_seg[seg] = whole ? make_int2(-1, -1) : make_int2(c, dec_cta_of(pc.seg_u0 + pc.npg - 1, T, C));
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32));   // scratch reuse
   } while (next_piece(pc));
+  }   // consumers
+
+  if constexpr (kCluster) {
+    if (cl_size > 1) {
+      // ---- merge of the cluster's states (log-sum-exp, as in the
+      // cross-warp combine): o = sum_c 2^(m_c - M) acc_c / sum_c 2^(m_c - M) l_c,
+      // lse = M + log2 sum_c 2^(m_c - M) le_c.  Each thread of the cluster
+      // takes float4 columns of the segment's rows.
+      cluster_sync();   // every CTA's state is in its shared memory
+      {
+        const int seg_in_b = cl_seg % nseg_b;
+        const int b = cl_seg / nseg_b;
+        const int kvh = seg_in_b / p.hgroups;
+        const int h0 = kvh * p.g + (seg_in_b % p.hgroups) * kDecHeadsPerSeg;
+        const int nh = min(kDecHeadsPerSeg, p.g - (seg_in_b % p.hgroups) * kDecHeadsPerSeg);
+        constexpr int kV4 = D / 4;
+        constexpr float kLn2 = 0.69314718055994530942f;
+        // item = (head r, float4 column l4), dealt round-robin over the
+        // cluster's CTAs first, so every CTA merges an equal part; each thread
+        // issues all of its remote loads (every CTA's abort flag and state)
+        // before using any of them, so an item costs one round trip
+        for (int it = cl_rank + cl_size * (int)threadIdx.x; it < nh * kV4;
+             it += cl_size * (int)blockDim.x) {
+          const int r = it / kV4, l4 = it % kV4;
+          float4 sc[16], oc[16];   // {m, l, l_exact, -} and the o columns of each CTA
+          int gave_up = 0;
+#pragma unroll
+          for (int q2 = 0; q2 < 16; ++q2) {
+            if (q2 < cl_size) {
+              gave_up |= dsmem_ld_s32(dsmem_addr(&abort_flag, (uint32_t)q2));
+              sc[q2] = dsmem_ld_f32x4(dsmem_addr(scratch + L::kXchS + 4 * r, (uint32_t)q2));
+              oc[q2] = dsmem_ld_f32x4(dsmem_addr(scratch + L::kXchO + r * D + 4 * l4, (uint32_t)q2));
+            }
+          }
+          if (gave_up) break;   // a CTA of the cluster stopped on a device error
+          float M = -INFINITY;
+#pragma unroll
+          for (int q2 = 0; q2 < 16; ++q2)
+            if (q2 < cl_size) M = fmaxf(M, sc[q2].x);
+          float ls = 0.f, le = 0.f;
+          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int q2 = 0; q2 < 16; ++q2) {
+            if (q2 < cl_size) {
+              // a CTA that saw no key (m = -inf) adds nothing
+              const float w = (sc[q2].x == -INFINITY) ? 0.f : fast_exp2(sc[q2].x - M);
+              ls += w * sc[q2].y;
+              le += w * sc[q2].z;
+              o4.x += w * oc[q2].x;
+              o4.y += w * oc[q2].y;
+              o4.z += w * oc[q2].z;
+              o4.w += w * oc[q2].w;
+            }
+          }
+          const float inv = ls > 0.f ? 1.f / ls : 0.f;
+          const size_t row = (size_t)b * p.Hq + h0 + r;
+          *reinterpret_cast<uint2*>(p.o + row * D + 4 * l4) =
+              make_uint2(pack_bf16x2(o4.x * inv, o4.y * inv), pack_bf16x2(o4.z * inv, o4.w * inv));
+          if (l4 == 0 && p.lse != nullptr) p.lse[row] = (M + fast_log2(le)) * kLn2;
+        }
+      }
+      cluster_sync();   // no CTA leaves while another still reads its shared memory
+    }
+  }
 }
 
 // Log-sum-exp merge of split segments' partials: o = sum_c 2^(lse_c - M) o_c /

@@ -10,6 +10,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/frt_attn.h"
@@ -27,21 +28,61 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxDevices = 64;
 
 // ------------------------------------------------------- device properties
+// Cluster-mode decode kernels (contiguous cache, no workspace), indexed by
+// [D == 128][two head tiles].
+using DecodeKernel = void (*)(CUtensorMap, CUtensorMap, DecodeParams);
+const DecodeKernel kClusterDecode[2][2] = {
+    {decode_splitkv_kernel<64, 1, false, true>, decode_splitkv_kernel<64, 2, false, true>},
+    {decode_splitkv_kernel<128, 1, false, true>, decode_splitkv_kernel<128, 2, false, true>}};
+constexpr size_t kClusterDecodeSmem[2][2] = {
+    {DecodeSmem<64, false, 1>::kBytes, DecodeSmem<64, false, 2>::kBytes},
+    {DecodeSmem<128, false, 1>::kBytes, DecodeSmem<128, false, 2>::kBytes}};
+constexpr int kClusterDecodeThreads[2] = {DecodeCfg<false, 1>::kThreads,
+                                          DecodeCfg<false, 2>::kThreads};
+
 struct DeviceInfo {
   int sm_count = 0;
   bool prefill_ok = false;   // register pool of the prefill launch covers its split
-  bool kernels_configured = false;
+  // clusters of c CTAs (index c, 1..16) of each cluster-mode decode kernel
+  // that the device holds at once; 0 where that size cannot be scheduled
+  int cluster_fit[2][2][17] = {};
+  // set (release) once every field above is final; read with acquire
+  std::atomic<bool> kernels_configured{false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
+
+// How many clusters of c CTAs of `kernel` the device holds at once, for
+// c = 1..16 (0 where that size cannot be scheduled).
+void cluster_fit(DecodeKernel kernel, size_t smem, int threads, int* fit) {
+  for (int c = 1; c <= 16; ++c) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();   // a refused size is not an error of the caller's
+      n = 0;
+    }
+    fit[c] = n;
+  }
+}
 
 frt_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FRT_ERR_CUDA;
   DeviceInfo& di = g_dev[dev];
-  if (!di.kernels_configured) {
+  if (!di.kernels_configured.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!di.kernels_configured) {
+    if (!di.kernels_configured.load(std::memory_order_relaxed)) {
       int sms = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FRT_ERR_CUDA;
@@ -89,7 +130,17 @@ frt_status device_info(DeviceInfo** out) {
         return FRT_ERR_CUDA;
       di.prefill_ok = true;
       for (const cudaFuncAttributes& a : fa) di.prefill_ok &= a.numRegs == kPfRegsLaunch;
-      di.kernels_configured = true;
+      for (int d = 0; d < 2; ++d)
+        for (int t = 0; t < 2; ++t) {
+          if (cudaFuncSetAttribute(kClusterDecode[d][t], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kClusterDecodeSmem[d][t]) != cudaSuccess ||
+              cudaFuncSetAttribute(kClusterDecode[d][t],
+                                   cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+            return FRT_ERR_CUDA;
+          cluster_fit(kClusterDecode[d][t], kClusterDecodeSmem[d][t], kClusterDecodeThreads[t],
+                      di.cluster_fit[d][t]);
+        }
+      di.kernels_configured.store(true, std::memory_order_release);
     }
   }
   *out = &di;
@@ -249,6 +300,8 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.max_pages = max_pages;
+  p.num_pages = block_table != nullptr ? (int)(cache_rows / ((uint64_t)Hkv * kDecPage)) : 0;
+  p.bad_row = (int)cache_rows;
   p.contig_len = contig_len;
   p.B = B;
   p.Hq = Hq;
@@ -303,6 +356,68 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
       launch_pdl((D == 128) ? decode_merge_kernel<128> : decode_merge_kernel<64>, dim3(merge_grid),
                  dim3(kMergeThreads), 0, stream, p);
   return err == cudaSuccess ? FRT_OK : FRT_ERR_CUDA;
+}
+
+// Single-token decode over a contiguous cache with no workspace: one cluster
+// of C CTAs per segment (sequence, KV head, group of <= 16 query heads), the
+// partial states merged through distributed shared memory.  C is the largest
+// cluster size whose grid (segments x C CTAs) the device holds in one wave,
+// with at most two CTAs per SM and one CTA per page.
+frt_status launch_decode_cluster(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int Skv, int D, float scale,
+                                 cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  frt_status st = device_info(&di);
+  if (st != FRT_OK) return st;
+  const int g = Hq / Hkv;
+  const int hgroups = (g + kDecHeadsPerSeg - 1) / kDecHeadsPerSeg;
+  const long long segments = (long long)B * Hkv * hgroups;
+  const int d128 = (D == 128) ? 1 : 0, two_tiles = (g > 8) ? 1 : 0;
+  const long long pages = (Skv + kDecPage - 1) / kDecPage;
+  const long long slots = (long long)kDecCtasPerSm * di->sm_count;
+  long long C = std::min<long long>(16, std::min(pages, slots / segments));
+  while (C > 1 && di->cluster_fit[d128][two_tiles][C] < segments) --C;
+  C = std::max<long long>(1, C);
+  if (segments * C > 0x7fffffffLL) return FRT_ERR_UNSUPPORTED;
+
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)B * Hkv * Skv;
+  const uint64_t dims[3] = {64, rows, (uint64_t)(D / 64)};
+  const uint64_t strides[2] = {(uint64_t)D * 2, 128};
+  const uint32_t box[3] = {64, (uint32_t)kDecPage, (uint32_t)(D / 64)};
+  if (!make_tmap(&tk, k, 3, dims, strides, box) || !make_tmap(&tv, v, 3, dims, strides, box))
+    return FRT_ERR_CUDA;
+  DecodeParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.contig_len = Skv;
+  p.bad_row = (int)rows;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.g = g;
+  p.hgroups = hgroups;
+  p.parts = (int)(segments * C);
+  p.scale_log2 = scale * kLog2e;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(segments * C));
+  cfg.blockDim = dim3(kClusterDecodeThreads[two_tiles]);
+  cfg.dynamicSmemBytes = kClusterDecodeSmem[d128][two_tiles];
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kClusterDecode[d128][two_tiles], tk, tv, p) == cudaSuccess
+             ? FRT_OK
+             : FRT_ERR_CUDA;
 }
 
 // Tiled tensor-core forward.  Contiguous K/V [B, Hkv, Skv, D] (paged == null),
@@ -379,6 +494,8 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.seq_lens = paged ? paged->seq_lens : nullptr;
   p.q_lens = paged ? paged->q_lens : nullptr;
   p.max_pages = paged ? paged->max_pages : 0;
+  p.num_pages = paged ? paged->num_pages : 0;
+  p.bad_row = paged ? paged->num_pages * Hkv * 16 : 0;
   const dim3 grid((unsigned)(B * Hq), (unsigned)n_blocks);
   auto* kernel = (paged == nullptr)
                      ? (D == 128 ? prefill_kernel<128, false> : prefill_kernel<64, false>)
@@ -397,7 +514,7 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 static __device__ __align__(256) unsigned char frt_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_noalloc_ptr[kMaxDevices];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];   // set once (release), read with acquire
 std::mutex g_noalloc_mutex;
 
 // Device address of this device's scratch (looked up on the first call made
@@ -405,16 +522,17 @@ std::mutex g_noalloc_mutex;
 frt_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FRT_ERR_CUDA;
-  if (g_noalloc_ptr[dev] == nullptr) {
+  void* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (ptr == nullptr) {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
-      void* ptr = nullptr;
+    ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (ptr == nullptr) {
       if (cudaGetSymbolAddress(&ptr, frt_noalloc_scratch) != cudaSuccess || ptr == nullptr)
         return FRT_ERR_CUDA;
-      g_noalloc_ptr[dev] = ptr;
+      g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
     }
   }
-  *out = g_noalloc_ptr[dev];
+  *out = ptr;
   return FRT_OK;
 }
 
@@ -478,8 +596,10 @@ frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void*
   if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
   if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
   if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
-  // the kernel's page prefix over the batch is 32-bit
-  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  // the kernel's page prefix over the batch and a sequence's token count are 32-bit
+  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31) ||
+      (uint64_t)max_pages_per_seq * page_size >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
   if (q != nullptr && B > 0) {
     if (k_pages == nullptr || v_pages == nullptr || o == nullptr ||
         seq_lens == nullptr || (block_table == nullptr && max_pages_per_seq > 0))
@@ -510,7 +630,9 @@ frt_status frt_attn_decode_paged_fp8(const void* q, const void* k_pages, const v
   if (page_size != kDecPage) return FRT_ERR_UNSUPPORTED;
   if (B > kDecMaxBatch) return FRT_ERR_UNSUPPORTED;
   if ((uint64_t)num_pages * Hkv * page_size >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
-  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31)) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)B * max_pages_per_seq >= (1ull << 31) ||
+      (uint64_t)max_pages_per_seq * page_size >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
   if (q != nullptr && B > 0) {
     if (k_pages == nullptr || v_pages == nullptr || o == nullptr || k_scale == nullptr ||
         v_scale == nullptr || seq_lens == nullptr ||
@@ -531,7 +653,28 @@ frt_status frt_attn_decode_paged_fp8(const void* q, const void* k_pages, const v
 
 frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int Hq, int Hkv, int Sq, int Skv, int D, int causal, float scale,
-                        void* workspace, size_t* workspace_bytes, cudaStream_t stream) {
+                        cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Skv < 0 ||
+      (causal != 0 && causal != 1) || !scale_ok(scale))
+    return FRT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FRT_ERR_UNSUPPORTED;
+  if ((uint64_t)B * Hkv * Skv >= (1ull << 31) || (uint64_t)B * Hq * Sq >= (1ull << 31))
+    return FRT_ERR_UNSUPPORTED;
+  if (B == 0 || Sq == 0) return FRT_OK;
+  if (q == nullptr || o == nullptr || (Skv > 0 && (k == nullptr || v == nullptr)))
+    return FRT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FRT_ERR_INVALID_ARG;
+  if (Sq == 1 && Skv > 0)
+    return launch_decode_cluster(q, k, v, o, lse, B, Hq, Hkv, Skv, D, scale, stream);
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream);
+}
+
+frt_status frt_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
+                           float scale, void* workspace, size_t* workspace_bytes,
+                           cudaStream_t stream) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Skv < 0 ||
       (causal != 0 && causal != 1) || !scale_ok(scale))
     return FRT_ERR_INVALID_ARG;

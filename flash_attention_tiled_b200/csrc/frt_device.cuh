@@ -18,6 +18,7 @@ namespace frt {
 enum : unsigned {
   kErrWaitTimeout = 1u << 0,   // an mbarrier wait exceeded its time limit
   kErrBadPlan = 1u << 1,       // inconsistent work plan (should be unreachable)
+  kErrBadPage = 1u << 2,       // a block-table entry outside [0, num_pages): read as zeros
 };
 
 // Defined here: the library is one translation unit (frt_attn.cu).
@@ -50,6 +51,54 @@ __device__ __forceinline__ bool elect_one() {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(pred));
   return pred != 0;
+}
+
+// ------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA of the cluster arrives (release) and waits
+// (acquire): shared-memory writes made before it are visible to the other
+// CTAs' reads after it.  Not the .aligned form, so a warp need not be
+// converged when it gets here.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release;\n\t"
+      "barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Address, in the cluster's shared window, of the same shared-memory
+// location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+
+// Loads from another CTA's shared memory.  Not volatile, so the compiler may
+// issue many before the first use; each depends on its address from
+// dsmem_addr (volatile), which keeps it after the cluster barrier before it.
+__device__ __forceinline__ int dsmem_ld_s32(uint32_t addr) {
+  int v;
+  asm("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t addr) {
+  float4 v;
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+      : "r"(addr));
+  return v;
 }
 
 // ----------------------------------------------------------------- mbarrier

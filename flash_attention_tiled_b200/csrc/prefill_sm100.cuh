@@ -86,6 +86,8 @@ struct PrefillParams {
   const int32_t* seq_lens;      // [B] cached tokens, the chunk included
   const int32_t* q_lens;        // [B] chunk lengths (<= Sq)
   int max_pages;
+  int num_pages;                // entries outside [0, num_pages) read row bad_row
+  int bad_row;                  // rows of the page pool's [rows, D] view (< 2^31): zeros
 };
 
 // kPaged: K and V come from a paged cache ([pages, Hkv, 16, D], 2D tensor
@@ -215,8 +217,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int npg = min(kPfBN / 16, (skv_b + 15) / 16 - j * (kPfBN / 16));
           int row = 0;
           if (lane < npg) {
+            // an entry outside [0, num_pages) is never an address: the copy
+            // starts past the pool's last row (zeros) and the error word
+            // records it; valid rows are below 2^31 (checked by the host)
             const int phys = p.block_table[(size_t)b * p.max_pages + j * (kPfBN / 16) + lane];
-            row = (phys * p.Hkv + kvh) * 16;
+            if ((unsigned)phys < (unsigned)p.num_pages) {
+              row = (int)(((long long)phys * p.Hkv + kvh) * 16);
+            } else {
+              row = p.bad_row;
+              raise_error(kErrBadPage);
+            }
           }
           if (lane == 0) mbar_arrive_expect_tx(&ring_full[slot], npg * kHalves * 16 * 128);
           __syncwarp();

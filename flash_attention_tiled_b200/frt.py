@@ -16,8 +16,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
-EXPORTS = ("frt_attn_fwd", "frt_attn_decode_paged", "frt_attn_decode_paged_noalloc",
-           "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8", "frt_attn_fwd_strided",
+EXPORTS = ("frt_attn_fwd", "frt_attn_fwd_ws", "frt_attn_decode_paged",
+           "frt_attn_decode_paged_noalloc", "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8", "frt_attn_fwd_strided",
            "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
            "frt_debug_fp8_decode", "frt_debug_wait_timeout", "frt_version")
 
@@ -38,7 +38,8 @@ def _load() -> ctypes.CDLL:
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_size_t)
-    lib.frt_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
+    lib.frt_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+    lib.frt_attn_fwd_ws.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
     lib.frt_attn_decode_paged.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I, P, Z, P]
     lib.frt_attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, P, I, I, P, P, I, I, I, I, F,
                                                   I, P]
@@ -144,10 +145,7 @@ def workspace(nbytes: int, device, stream_handle: int) -> torch.Tensor:
     return ws
 
 
-def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
-             scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, return_lse: bool = True):
-    """o, lse = attention(q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D]) with bf16 tensors."""
+def _fwd_args(q, k, v, causal, scale, out, lse, return_lse):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, torch.bfloat16, 4)
     B, Hq, Sq, D = q.shape
@@ -163,18 +161,41 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    return (B, Hq, Hkv, Sq, Skv, D), scale, out, lse
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, return_lse: bool = True):
+    """o, lse = attention(q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D]) with bf16 tensors
+    (frt_attn_fwd: no workspace; Sq = 1 runs the cluster-merged decode)."""
+    (B, Hq, Hkv, Sq, Skv, D), scale, out, lse = _fwd_args(q, k, v, causal, scale, out, lse,
+                                                          return_lse)
+    _check("frt_attn_fwd", _lib.frt_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
+                                             Hq, Hkv, Sq, Skv, D, int(causal), scale,
+                                             _stream(q.device)))
+    return out, lse
+
+
+def attn_fwd_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                scale: float | None = None, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None, return_lse: bool = True):
+    """attn_fwd through frt_attn_fwd_ws: Sq = 1 runs the split-KV decode with a
+    workspace (from this module's per-stream buffers) and its merge kernel."""
+    (B, Hq, Hkv, Sq, Skv, D), scale, out, lse = _fwd_args(q, k, v, causal, scale, out, lse,
+                                                          return_lse)
     stream = _stream(q.device)
     need = ctypes.c_size_t(0)
-    _check("frt_attn_fwd", _lib.frt_attn_fwd(None, None, None, None, None, B, Hq, Hkv, Sq, Skv,
-                                             D, int(causal), scale, None, ctypes.byref(need),
-                                             stream))
+    _check("frt_attn_fwd_ws", _lib.frt_attn_fwd_ws(None, None, None, None, None, B, Hq, Hkv, Sq,
+                                                   Skv, D, int(causal), scale, None,
+                                                   ctypes.byref(need), stream))
     ws = None
     if need.value > 0:
         ws = workspace(need.value, q.device, stream.value)
         need = ctypes.c_size_t(ws.numel())
-    _check("frt_attn_fwd", _lib.frt_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
-                                             Hq, Hkv, Sq, Skv, D, int(causal), scale, _ptr(ws),
-                                             ctypes.byref(need), stream))
+    _check("frt_attn_fwd_ws", _lib.frt_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                   _ptr(lse), B, Hq, Hkv, Sq, Skv, D, int(causal),
+                                                   scale, _ptr(ws), ctypes.byref(need), stream))
     return out, lse
 
 

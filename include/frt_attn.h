@@ -69,8 +69,12 @@ typedef enum {
 } frt_status;
 
 /*
- * frt_attn_fwd -- attention over a contiguous KV tensor (prefill, chunked
- * prefill, cross attention and single-token decode).
+ * frt_attn_fwd -- attention over a contiguous KV tensor (prefill, cross
+ * attention and single-token decode).  The calling convention is the
+ * plugin's of the "Analysis of TensorRT's low-level support for
+ * FlashAttention" page (plugin sketch, enqueue): Q, K, V and O pointers, head
+ * counts, query and key lengths, head dimension and the caller's stream; the
+ * call returns 0 (FRT_OK) once the work is queued.  It needs no workspace.
  *
  *   q   [B, Hq,  Sq,  D] bf16      k, v  [B, Hkv, Skv, D] bf16
  *   o   [B, Hq,  Sq,  D] bf16      lse   [B, Hq, Sq] fp32, may be NULL
@@ -78,19 +82,35 @@ typedef enum {
  *   (1/sqrt(D) in the usual model).
  *
  * Sq > 1 runs the tiled tensor-core kernel (128-query tiles, 128-key tiles,
- * fully masked key tiles skipped).  Sq == 1 runs the split-KV decode kernel
- * over the contiguous cache; that path needs a workspace like
- * frt_attn_decode_paged (same rules) and takes it from `workspace`.
- * Size query: a call with q == NULL only writes the workspace size to
- * *workspace_bytes (0 when Sq > 1) and returns FRT_OK; workspace and
- * workspace_bytes may be NULL on real calls that need none (Sq > 1).
- * B, Sq or Skv may be 0 (nothing to attend: o = 0, lse = -inf where rows
- * exist).
+ * fully masked key tiles skipped).  Sq == 1 runs the decode kernel in
+ * cluster mode: each (sequence, KV head) is streamed by a cluster of up to
+ * 16 CTAs whose partial results are merged by log-sum-exp inside the
+ * cluster (distributed shared memory), in one launch and with no scratch in
+ * global memory.  For a very long cache with few KV heads (fewer than about
+ * 16 sequences x KV heads) frt_attn_fwd_ws spreads the keys over more of the
+ * GPU.  B, Sq or Skv may be 0 (nothing to attend: o = 0, lse = -inf where
+ * rows exist).
  */
 FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int Hq, int Hkv, int Sq, int Skv, int D, int causal,
-                        float scale, void* workspace, size_t* workspace_bytes,
-                        cudaStream_t stream);
+                        float scale, cudaStream_t stream);
+
+/*
+ * frt_attn_fwd_ws -- frt_attn_fwd with a caller workspace, for single-token
+ * decode over a long contiguous cache: Sq == 1 runs the split-KV decode of
+ * frt_attn_decode_paged (any number of partitions per sequence, then the
+ * log-sum-exp merge kernel), which keeps the whole GPU busy even for one
+ * sequence with one KV head.  Sq > 1 is frt_attn_fwd.
+ * Size query: a call with q == NULL only writes the workspace size to
+ * *workspace_bytes (0 when Sq > 1) and returns FRT_OK; workspace and
+ * workspace_bytes may be NULL on real calls that need none (Sq > 1).  The
+ * workspace rules are those of frt_attn_decode_paged.  Sq == 1 limits B to
+ * 1024.
+ */
+FRT_API frt_status frt_attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
+                                   float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                                   int causal, float scale, void* workspace,
+                                   size_t* workspace_bytes, cudaStream_t stream);
 
 /*
  * frt_attn_decode_paged -- one query token per sequence over a paged KV
@@ -131,15 +151,19 @@ FRT_API frt_status frt_attn_fwd(const void* q, const void* k, const void* v, voi
  * Both start by waiting for the work before them in the stream, so the call
  * is ordered like any other stream operation.
  *
- * Block-table entries outside [0, num_pages) read zeros (the copy engine's
- * bounds), never out-of-bounds memory.  Tail slots of the last page of a
- * sequence may hold anything, NaN included: they never reach o.
+ * A block-table entry outside [0, num_pages) that a sequence uses is never
+ * turned into an address: the kernel checks it before issuing the copy,
+ * reads that page as all zeros (keys and values 0) and sets bit 2 of the
+ * device error word (frt_read_device_error).  The other sequences' results
+ * are unaffected.  Tail slots of the last page of a sequence may hold
+ * anything, NaN included: they never reach o.
  *
- * Size limit: the pages of all sequences together, B * max_pages_per_seq,
- * must stay below 2^31 (FRT_ERR_UNSUPPORTED otherwise), since the kernel
- * counts pages in 32 bits.  Sequences may share physical pages, so this
- * limits the block table, not the cache.  Reaching it takes a block table
- * of 8 GB or more.
+ * Size limits (FRT_ERR_UNSUPPORTED otherwise), since the kernel counts pages
+ * and tokens in 32 bits: the pages of all sequences together,
+ * B * max_pages_per_seq, below 2^31; a sequence's token bound,
+ * max_pages_per_seq * page_size, below 2^31; and the cache's rows,
+ * num_pages * Hkv * page_size, below 2^31.  Sequences may share physical
+ * pages, so the first limits the block table, not the cache.
  */
 FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                                  const int32_t* block_table, int max_pages_per_seq,
@@ -171,7 +195,9 @@ FRT_API frt_status frt_attn_decode_paged(const void* q, const void* k_pages, con
  *   page_size   16
  * Runs the tiled tensor-core kernel with K/V tiles gathered page by page
  * through the block table.  Needs no workspace.  Tail slots of a sequence's
- * last page may hold anything, NaN included.
+ * last page may hold anything, NaN included.  A block-table entry outside
+ * [0, num_pages) is handled as in frt_attn_decode_paged: checked before any
+ * copy, read as a page of zeros, reported in bit 2 of the error word.
  *
  * Size limit: max_pages_per_seq * 16 must stay below 2^31
  * (FRT_ERR_UNSUPPORTED otherwise), since a sequence's length bound is
@@ -297,7 +323,9 @@ FRT_API frt_status frt_attn_merge_lse(const float* o_parts, const float* lse_par
  * frt_read_device_error -- read and clear the library's device-side error
  * word on the current device (synchronises that device).  0 means no kernel
  * gave up; bit 0 = an internal wait timed out (the kernel returned without
- * finishing its outputs).  Returns FRT_ERR_CUDA if the read itself failed.
+ * finishing its outputs); bit 2 = a block-table entry outside [0, num_pages)
+ * was met (that page was read as zeros, nothing outside the cache was
+ * touched).  Returns FRT_ERR_CUDA if the read itself failed.
  */
 FRT_API frt_status frt_read_device_error(unsigned* flags);
 

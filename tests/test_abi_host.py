@@ -38,8 +38,24 @@ Z = ctypes.c_size_t
 
 def _fwd(B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64, causal=0, scale=0.125, query=True):
     need = Z(0)
-    return frt.lib().frt_attn_fwd(NULL, NULL, NULL, NULL, NULL, B, Hq, Hkv, Sq, Skv, D, causal,
-                                  scale, NULL, ctypes.byref(need), NULL), need.value
+    return frt.lib().frt_attn_fwd_ws(NULL, NULL, NULL, NULL, NULL, B, Hq, Hkv, Sq, Skv, D, causal,
+                                     scale, NULL, ctypes.byref(need), NULL), need.value
+
+
+def _fwd14(q=NULL, k=NULL, v=NULL, o=NULL, lse=NULL, B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64,
+           causal=0, scale=0.125):
+    return frt.lib().frt_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, NULL)
+
+
+def test_fwd_has_the_plugin_signature():
+    # frt_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, causal, scale, stream): the
+    # plugin convention of the TensorRT analysis page, no workspace arguments
+    text = open(os.path.join(ROOT, "include", "frt_attn.h")).read()
+    m = re.search(r"FRT_API\s+frt_status\s+frt_attn_fwd\s*\(([^)]*)\)", text)
+    params = [re.findall(r"(\w+)\s*$", p.strip())[0] for p in m.group(1).split(",")]
+    assert params == ["q", "k", "v", "o", "lse", "B", "Hq", "Hkv", "Sq", "Skv", "D", "causal",
+                      "scale", "stream"]
+    assert len(frt.lib().frt_attn_fwd.argtypes) == 14
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -57,6 +73,7 @@ def _fwd(B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64, causal=0, scale=0.125, query=True)
 def test_fwd_rejects(kw, code):
     rc, _ = _fwd(**kw)
     assert rc == code
+    assert _fwd14(**kw) == code      # the workspace-free entry checks the same
 
 
 def test_fwd_prefill_needs_no_workspace():
@@ -170,8 +187,11 @@ ODD = ctypes.c_void_p((1 << 20) + 2)   # 2-byte aligned only
 
 def _fwd_call(q=A16, k=A16, v=A16, o=A16, lse=NULL, B=1, Hq=2, Hkv=2, Sq=4, Skv=4, D=64):
     need = Z(0)
-    return frt.lib().frt_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, 0, 0.125, NULL,
-                                  ctypes.byref(need), NULL)
+    rc = frt.lib().frt_attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, 0, 0.125, NULL,
+                                   ctypes.byref(need), NULL)
+    rc14 = _fwd14(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D)
+    assert rc14 == rc, (rc14, rc)
+    return rc
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -182,6 +202,7 @@ def _fwd_call(q=A16, k=A16, v=A16, o=A16, lse=NULL, B=1, Hq=2, Hkv=2, Sq=4, Skv=
     (dict(v=ODD), 1),
     (dict(lse=ODD), 1),
     (dict(Sq=1, q=ODD), 1),                     # the decode path checks the same
+    (dict(Sq=1, o=NULL), 1),
     (dict(B=1 << 16, Hq=1 << 8, Hkv=1 << 8, Sq=1 << 8, Skv=1), 2),   # 2^32 query rows
 ])
 def test_fwd_real_call_rejects(kw, code):
@@ -290,3 +311,8 @@ def test_page_count_limits_are_checked():
                                                10, NULL, NULL, 1024, 8, 2, 128, 0.1, 4, NULL,
                                                ctypes.byref(need), NULL) == 2
     assert _prefill_paged(maxp=1 << 27) == 2
+    # a sequence's token bound max_pages_per_seq * 16 >= 2^31 (paged decode)
+    assert _paged_call(B=1, maxp=1 << 27) == 2
+    assert frt.lib().frt_attn_decode_paged_fp8(NULL, NULL, NULL, NULL, NULL, NULL, 1 << 27, NULL, 16,
+                                               10, NULL, NULL, 1, 8, 2, 128, 0.1, 4, NULL,
+                                               ctypes.byref(need), NULL) == 2

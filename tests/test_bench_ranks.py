@@ -90,3 +90,12 @@ def test_reference_line_shape(monkeypatch):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "step/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_the_gpu_arms_step_counts():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reference_plan(20, 5) == (20, 5)      # the driver's K and W: exactly those
+    assert bench.reference_plan(3, 3) == (3, 3)
+    timed, untimed = bench.reference_plan(2000, 20)   # the default K would take hours
+    assert 1 <= timed and timed + untimed <= bench.REF_BUDGET_S // bench.REF_STEP_S_EST

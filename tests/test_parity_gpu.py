@@ -2,9 +2,9 @@
 
 Bar (all outputs are bf16 from fp32 accumulation): max |o - o_ref| <= 1e-2,
 mean |o - o_ref| <= 1e-3, max |lse - lse_ref| <= 1e-3; index work (which
-page, which slot) bit-exact.  The five named workloads run at full size;
-where the oracle would take too long (the 4k prefill) it checks sampled rows,
-computed one by one, of the very launch the benchmark times.
+page, which slot) bit-exact.  The five named workloads run at full size and are
+compared element by element, each with the launch configuration the
+benchmark times.
 """
 import ctypes
 import math
@@ -67,33 +67,30 @@ def test_tiny_causal(frt):
     _no_device_error(frt)
 
 
-def test_gqa_decode_contiguous(frt):
+@pytest.mark.parametrize("entry", ["attn_fwd", "attn_fwd_ws"])
+def test_gqa_decode_contiguous(frt, entry):
+    # attn_fwd: the cluster-merged decode (what the benchmark times);
+    # attn_fwd_ws: the split-KV decode with a workspace and its merge kernel
     w = inputs.WORKLOADS["gqa_decode_4k"]
     x = inputs.make(w)
     d = _dev(x)
-    o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=False, scale=w.scale)
+    o, lse = getattr(frt, entry)(d["q"], d["k"], d["v"], causal=False, scale=w.scale)
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], False, w.scale)
     _compare(o, o_ref, lse, lse_ref, "gqa_decode_4k")
     _no_device_error(frt)
 
 
-def test_llama3_prefill_sampled_rows(frt):
+def test_llama3_prefill_full(frt):
+    # every element of the 32 x 4096 x 128 output and every LSE of the launch
+    # the benchmark times, against the oracle's full fp64 score matrices
     w = inputs.WORKLOADS["llama3_8b_prefill_4k"]
     x = inputs.make(w)
     d = _dev(x)
     o, lse = frt.attn_fwd(d["q"], d["k"], d["v"], causal=True, scale=w.scale)
     torch.cuda.synchronize()
-    gen = np.random.default_rng(7)
-    rows = []
-    for h in (0, 5, 17, 31):
-        base = h * w.Sq
-        rows += [base + i for i in (0, 1, 2, 3, 127, 128, 129, 255, 1000, 2047, 2048, 4094, 4095)]
-    rows += list(gen.integers(0, w.Hq * w.Sq, size=200))
-    rows = np.array(sorted(set(int(r) for r in rows)), dtype=np.int64)
-    o_ref, lse_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], True, w.scale, rows)
-    _compare(o.reshape(-1, w.D)[torch.from_numpy(rows).cuda()], o_ref,
-             lse.reshape(-1)[torch.from_numpy(rows).cuda()], lse_ref, "prefill sampled")
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], True, w.scale)
+    _compare(o, o_ref, lse, lse_ref, "llama3 prefill (all rows)")
     # properties that hold at any size: row 0 of every head is v[0] exactly,
     # and every output lies in the convex hull of the values it attends
     kvh = torch.arange(w.Hq, device="cuda") // (w.Hq // w.Hkv)
@@ -207,11 +204,12 @@ def test_decode_edge(frt, case):
     _no_device_error(frt)
 
 
-def test_decode_contiguous_ragged(frt):
+@pytest.mark.parametrize("entry", ["attn_fwd", "attn_fwd_ws"])
+def test_decode_contiguous_ragged(frt, entry):
     for Skv in (1, 7, 16, 100, 1025):
         x = inputs.dense(2, 8, 2, 1, Skv, 128, seed=Skv)
         d = _dev(x)
-        o, lse = frt.attn_fwd(d["q"], d["k"], d["v"])
+        o, lse = getattr(frt, entry)(d["q"], d["k"], d["v"])
         torch.cuda.synchronize()
         o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], False, 1 / math.sqrt(128))
         _compare(o, o_ref, lse, lse_ref, f"contiguous decode Skv={Skv}")
