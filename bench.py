@@ -522,7 +522,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, shuffled page tables)",
         "config": {"workload": WORKLOAD, "global_batch": None, "seq_len": 4096,
                    "parallelism": f"replicas x{world}",
-                   "timing": "step = one CUDA graph of the four calls, replayed K times; "
+                   "timing": "step = one CUDA graph of the five calls, replayed K times; "
                              "per-call times: a graph of 20 x (L2 flush, call) minus a "
                              "graph of 20 flushes, divided by 20",
                    "l2": "step working set ~0.9 GB > 126 MB L2 and every call's inputs are "
@@ -536,7 +536,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": sum(Step.LAUNCHES[n] for n in names) * args.steps * world,   # all ranks
         "clocks": dict(sampler.summary(), window=(
-            f"{PREROLL_S:.0f} s of untimed step replays ({preroll} steps) immediately before "
+            f"{PREROLL_S:.1f} s of untimed step replays ({preroll} steps) immediately before "
             f"the timed region, and the timed region")),
     }
     return line

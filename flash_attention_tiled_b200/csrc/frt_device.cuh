@@ -364,34 +364,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x on the FMA pipe for a pair of fp32 values, to take part of the
-// exponentials off the MUFU unit.  Method: Cody-Waite style range reduction
-// x = j + f with j = round(x) (added to 1.5 * 2^23 so that the integer lands
-// in the low mantissa bits) and f in [-1/2, 1/2], a cubic for 2^f whose
-// coefficients were fitted for this library by a Remez exchange on the
-// relative error (max relative error 7.5e-5, far below a bf16 half-ulp of
-// 2^-9), and 2^j applied by an integer add into the exponent field.
-// Valid for x in [-125, 126]; callers clamp below at -125 (2^-125 is ~0 for
-// every use here).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t neg_one = f2_pack(-1.0f, -1.0f);
-  const uint64_t t = f2_add(x2, magic);            // integer part in the low bits
-  const uint64_t j = f2_add(t, neg_magic);         // round(x) as a float
-  const uint64_t f = f2_fma(j, neg_one, x2);       // x - round(x)
-  uint64_t q = f2_fma(f2_pack(0.055171669f, 0.055171669f), f,
-                      f2_pack(0.24261112f, 0.24261112f));
-  q = f2_fma(q, f, f2_pack(0.69326099f, 0.69326099f));
-  q = f2_fma(q, f, f2_pack(0.99992807f, 0.99992807f));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t, t0, t1);
-  const float y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  const float y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-  return f2_pack(y0, y1);
-}
-
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

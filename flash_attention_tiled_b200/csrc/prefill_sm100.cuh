@@ -10,8 +10,12 @@
 // optimisation".  Key tiles that the causal mask hides completely are never
 // loaded or multiplied.
 //
-// One CTA owns two 128-row query tiles (A = rows 0-127, B = rows 128-255 of a
-// 256-row block of one head) that share every K/V tile.  Tensor memory holds
+// One CTA owns two 128-row query tiles A and B that share every K/V tile.
+// When a KV head serves an even number of query heads (GQA with g even, MQA)
+// the tiles are the same 128 rows of two query heads of one KV head, so each
+// K/V tile staged in shared memory serves two heads of its group (the MQA/GQA
+// head sharing of the "FlashRT-HF-kernels" page); otherwise (g odd, e.g. MHA)
+// they are rows 0-127 and 128-255 of a 256-row block of one head.  Tensor memory holds
 // S_A, S_B (128 fp32 columns each) and O_A, O_B (D columns each).  P_X is
 // written as bf16 into its own shared-memory tile (the A operand of
 // O_X += P_X.V), so S_X is free as soon as the softmax has read it: S_X(j+1)
@@ -50,9 +54,6 @@ constexpr int kPfRegsSoftmax = 208;    // warpgroups 1, 2 after setmaxnreg.inc
 static_assert(128 * kPfRegsProducer + 256 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
               "register split must fit in the launch's register pool");
 constexpr float kPfRescaleThreshold = 8.0f;   // log2 units
-// Every kPfPolyEvery-th pair of exponentials is computed on the FMA pipe
-// (exp2_poly_x2) instead of MUFU; 0 keeps all of them on MUFU.
-constexpr int kPfPolyEvery = 0;
 
 template <int D>
 struct PrefillSmem {
@@ -78,7 +79,9 @@ struct PrefillSmem {
 
 struct PrefillParams {
   float* lse;          // [B, Hq, Sq] or nullptr
-  int B, Hq, Hkv, g, Sq, Skv, causal, n_blocks;   // n_blocks = ceil(Sq / 256)
+  int B, Hq, Hkv, g, Sq, Skv, causal, n_blocks;   // n_blocks = ceil(Sq / block rows)
+  int head_pairs;      // 1: the two tiles are two heads (g even), 128-row blocks;
+                       // 0: the two tiles are two row halves of one head, 256-row blocks
   float scale_log2;
   // paged K/V (chunked prefill): Sq is the padded chunk length max_q, the
   // per-sequence chunk and context lengths are read on the device
@@ -129,13 +132,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- block coordinates (heaviest causal blocks are scheduled first)
-  const int bh = blockIdx.x;                 // b * Hq + hq
+  // ---- block coordinates (heaviest causal blocks are scheduled first).
+  // Tile t covers query head hq0 + t * dh, rows q_blk + t * dr .. + 127.
+  const int heads_per_cta = p.head_pairs ? 2 : 1;
+  const int blk_rows = p.head_pairs ? kPfBM : kPfRows;
+  const int dh = p.head_pairs ? 1 : 0, dr = p.head_pairs ? 0 : kPfBM;
+  const int hgrp = p.Hq / heads_per_cta;
   const int blk = p.causal ? (p.n_blocks - 1 - (int)blockIdx.y) : (int)blockIdx.y;
-  const int b = bh / p.Hq, hq = bh % p.Hq;
-  const int kvh = hq / p.g;
+  const int b = (int)blockIdx.x / hgrp;
+  const int hq0 = ((int)blockIdx.x % hgrp) * heads_per_cta;   // first query head
+  const int kvh = hq0 / p.g;                 // (g even: both heads share it)
   // Q, O, K and V maps are 4D (d, token, head, batch), so any strides work
-  const int q_blk = blk * kPfRows;           // first query row of tile A
+  const int q_blk = blk * blk_rows;          // first query row of tile A
   // this sequence's chunk (query) length and context (key) length
   int sq_b = p.Sq, skv_b = p.Skv;
   if (kPaged) {
@@ -143,7 +151,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     skv_b = min(max(p.seq_lens[b], 0), p.max_pages * 16);
   }
   const int off = skv_b - sq_b;              // bottom-right causal alignment
-  const int q_last = min(q_blk + kPfRows - 1, sq_b - 1);
+  const int q_last = min(q_blk + blk_rows - 1, sq_b - 1);
   const int n_kv_all = (skv_b + kPfBN - 1) / kPfBN;
   int n_kv = q_last < q_blk ? 0 : n_kv_all;  // a block wholly in the padding has no work
   if (p.causal && n_kv > 0) {
@@ -193,7 +201,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int h = 0; h < kHalves; ++h)
             tma_load_4d(sq + t * L::kTileBytes + h * L::kHalfBytes, &tm_q, q_full, h * 64,
-                        q_blk + t * kPfBM, hq, b);
+                        q_blk + t * dr, hq0 + t * dh, b);
       }
       int slot = 0;
       uint32_t phase = 0;
@@ -351,7 +359,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int t = (warp >> 2) - 1;                // query tile of this warpgroup
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // row within the tile
-    const int q0 = q_blk + t * kPfBM;             // first query row of the tile
+    const int q0 = q_blk + t * dr;                // first query row of the tile
+    const int hq = hq0 + t * dh;                  // query head of the tile
     const int qi = q0 + r;                        // query index
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_addr = lane_addr + L::col_s(t);
@@ -446,13 +455,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int c = c8 + 2 * q;
             float x0, x1, e0, e1;
             f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, ref2), x0, x1);
-            constexpr int kEvery = kPfPolyEvery > 0 ? kPfPolyEvery : 1;
-            if (kPfPolyEvery > 0 && (c / 2) % kEvery == kEvery - 1) {
-              f2_unpack(exp2_poly_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), e0, e1);
-            } else {
-              e0 = fast_exp2(x0);
-              e1 = fast_exp2(x1);
-            }
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
             w[q] = pack_bf16x2(e0, e1);
             const uint64_t wr = f2_pack(__uint_as_float(w[q] << 16),
                                         __uint_as_float(w[q] & 0xffff0000u));
@@ -517,7 +521,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       if (p.lse != nullptr && qi < p.Sq) {   // padding rows get -inf
         const float lse2 = (any_key && l_exact > 0.f) ? m_ref + fast_log2(l_exact) : -INFINITY;
-        p.lse[(size_t)bh * p.Sq + qi] = lse2 * 0.69314718055994530942f;
+        p.lse[((size_t)b * p.Hq + hq) * p.Sq + qi] = lse2 * 0.69314718055994530942f;
       }
       fence_proxy_async_smem();
     }

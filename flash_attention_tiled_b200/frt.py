@@ -17,8 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt_attn.so")
 
 EXPORTS = ("frt_attn_fwd", "frt_attn_fwd_ws", "frt_attn_decode_paged",
-           "frt_attn_decode_paged_noalloc", "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8", "frt_attn_fwd_strided",
-           "frt_attn_merge_lse", "frt_read_device_error", "frt_debug_exp2_poly",
+           "frt_attn_decode_paged_noalloc", "frt_attn_prefill_paged", "frt_attn_decode_paged_fp8",
+           "frt_attn_fwd_strided", "frt_attn_merge_lse", "frt_read_device_error",
            "frt_debug_fp8_decode", "frt_debug_wait_timeout", "frt_version")
 
 STATUS = {0: "FRT_OK", 1: "FRT_ERR_INVALID_ARG", 2: "FRT_ERR_UNSUPPORTED",
@@ -47,7 +47,6 @@ def _load() -> ctypes.CDLL:
     lib.frt_attn_prefill_paged.argtypes = [P, P, P, P, I, P, P, I, I, P, P, I, I, I, I, I, I, F,
                                            P]
     lib.frt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
-    lib.frt_debug_exp2_poly.argtypes = [P, P, I, P]
     lib.frt_attn_decode_paged_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, P, P, I, I, I, I, F, I,
                                               P, Z, P]
     lib.frt_debug_fp8_decode.argtypes = [P, P, I, P]
@@ -127,6 +126,13 @@ def _same_device(device, **tensors):
 # whatever its shape.  It grows in powers of two when a call needs more; an
 # outgrown buffer is kept alive (a captured CUDA graph may still use it), so
 # all buffers together hold less than twice the largest need.
+#
+# The key is the raw stream handle.  Streams from torch's pool are never
+# destroyed, so there a handle always names the same stream.  Two cases are
+# the caller's to order: an external stream destroyed and replaced by a new
+# one with the same handle (synchronise the old one first), and a CUDA graph
+# captured on stream A replayed on another stream while eager calls run on A
+# (the graph holds A's buffer; order the replay after A's calls).
 _workspaces: dict = {}
 _retired: list = []
 
@@ -427,15 +433,6 @@ def merge_lse(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor 
         _ptr(o_parts), _ptr(lse_parts), S, B, Hq, D, _ptr(out), _ptr(lse),
         _stream(o_parts.device)))
     return out, lse
-
-
-def debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
-    """The library's FMA-pipe 2^x evaluated on a CUDA float32 tensor (diagnostic)."""
-    _need(x, "x", torch.float32, x.dim())
-    y = torch.empty_like(x)
-    _check("frt_debug_exp2_poly", _lib.frt_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(),
-                                                           _stream(x.device)))
-    return y
 
 
 def read_device_error() -> int:

@@ -284,7 +284,9 @@ FRT_API frt_status frt_attn_fwd_strided(const void* q, const void* k, const void
  * frt_attn_decode_paged: [num_pages, Hkv, page_size, D] uint8.  An element
  * of KV head h stands for code * k_scale[h] (keys) or code * v_scale[h]
  * (values); every other argument means what it means for
- * frt_attn_decode_paged, and the workspace size query is the same.
+ * frt_attn_decode_paged, and the workspace size query is the same, except
+ * that num_splits = 0 means two partitions per SM (296 on a 148-SM B200):
+ * with one byte per element the kernel's arithmetic, not HBM, sets its pace.
  *   k_scale, v_scale  [Hkv] fp32 on the device, finite, 4-byte aligned
  *   D                 128 only (FRT_ERR_UNSUPPORTED otherwise)
  * The kernel converts codes to f16 (exact), multiplies q.k in f16 with fp32
@@ -338,15 +340,6 @@ FRT_API frt_status frt_read_device_error(unsigned* flags);
  * usable.  returned: one device int32, 16-byte aligned.
  */
 FRT_API frt_status frt_debug_wait_timeout(int* returned, cudaStream_t stream);
-
-/*
- * frt_debug_exp2_poly -- diagnostic: y[i] = the library's FMA-pipe 2^x for
- * x[i] (device arrays of n floats; inputs below -125 are clamped there).
- * The prefill kernel's softmax can compute part of its exponentials this way
- * (a compile-time option, off in this build); tests compare it with CUDA's
- * exp2f.  Not part of the attention path.
- */
-FRT_API frt_status frt_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 
 /*
  * frt_debug_fp8_decode -- diagnostic: y[i] = the value of e4m3 code codes[i]

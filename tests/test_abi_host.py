@@ -297,9 +297,6 @@ def test_merge_real_call_rejects_misaligned():
 def test_diagnostic_entries_check_their_arguments():
     lib = frt.lib()
     assert lib.frt_read_device_error(None) == 1
-    assert lib.frt_debug_exp2_poly(NULL, NULL, -1, NULL) == 1
-    assert lib.frt_debug_exp2_poly(NULL, NULL, 0, NULL) == 0
-    assert lib.frt_debug_exp2_poly(NULL, NULL, 4, NULL) == 1
 
 
 def test_page_count_limits_are_checked():
