@@ -68,6 +68,11 @@ struct DecodeCfg {
 constexpr int kDecCtasPerSm = 2;
 constexpr long long kDecInFlightBytes = 18ll << 20;
 constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
+// The producer reads block-table entries for 32 pages at a time (one per
+// lane) and hands them out stage by stage, so a stage must divide 32 pages.
+static_assert(32 % DecodeCfg<false, 1>::kStagePages == 0 && 32 % DecodeCfg<false, 2>::kStagePages == 0 &&
+                  32 % DecodeCfg<true, 1>::kStagePages == 0 && 32 % DecodeCfg<true, 2>::kStagePages == 0,
+              "stages of whole windows");
 constexpr int kDecMaxBatch = 1024;    // prefix table held in shared memory
 
 struct DecodeParams {
@@ -327,12 +332,16 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
     bool ok = true;
     do {
       const int kvh = pc.seg_in_b / p.hgroups;
-      for (int pb = pc.pg0; pb < pc.pg1 && ok; pb += kDecStagePages) {
-        const int n = min(kDecStagePages, pc.pg1 - pb);
-        // row of the page's first token in the [rows, D] view of the cache
-        int row = 0;
-        if (lane < n) {
-          const int page = pb + lane;
+      // Rows (first token of each page in the [rows, D] view of the cache) of
+      // the next 32 pages of this piece, one per lane, so the block table is
+      // read in one round trip per 32 pages instead of one per stage and the
+      // ring's first stages are issued back to back.
+      int win0 = pc.pg0, win_row = 0;
+      auto load_window = [&](int first) {
+        win0 = first;
+        win_row = 0;
+        const int page = first + lane;
+        if (page < pc.pg1) {
           if (p.block_table != nullptr) {
             // An entry outside [0, num_pages) is never used as an address:
             // the copy starts past the cache's last row, so the page reads as
@@ -340,16 +349,23 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // num_pages * Hkv * 16 < 2^31 (checked by the host).
             const int phys = p.block_table[(size_t)pc.b * p.max_pages + page];
             if ((unsigned)phys < (unsigned)p.num_pages) {
-              row = (int)(((long long)phys * p.Hkv + kvh) * kDecPage);
+              win_row = (int)(((long long)phys * p.Hkv + kvh) * kDecPage);
             } else {
-              row = p.bad_row;
+              win_row = p.bad_row;
               raise_error(kErrBadPage);
             }
           } else {
-            row = (int)(((long long)pc.b * p.Hkv + kvh) * p.contig_len + (long long)page * kDecPage);
+            win_row = (int)(((long long)pc.b * p.Hkv + kvh) * p.contig_len +
+                            (long long)page * kDecPage);
           }
         }
-        ok = mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag);
+      };
+      load_window(pc.pg0);
+      for (int pb = pc.pg0; pb < pc.pg1 && ok; pb += kDecStagePages) {
+        const int n = min(kDecStagePages, pc.pg1 - pb);
+        if (pb + n > win0 + 32) load_window(pb);   // (a stage never straddles two windows)
+        const int row = __shfl_sync(0xffffffffu, win_row, (pb - win0 + lane) & 31);
+        ok = mbar_wait_warp(&empty_bar[stage], phase ^ 1u, &abort_flag);
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], n * 2 * L::kPageBytes);
         __syncwarp();
