@@ -894,9 +894,9 @@ __global__ void __launch_bounds__(kMergeThreads, 2) decode_merge_kernel(const De
   __shared__ float4 red[kGroups][kV];
   __shared__ float red_m[kGroups], red_s[kGroups];
   __shared__ int list[kMergeThreads];
+  __shared__ int2 range[kMergeThreads];         // CTAs holding the row's pieces
+  __shared__ int prefix[kDecMaxBatch + 1];      // page prefix over the batch
   __shared__ int nlist, max_parts;
-  griddep_wait();   // the streaming kernel's partials and segment table
-  griddep_launch_dependents();
 
   const int t = threadIdx.x, grp = t / kV, l = t % kV;
   const int nseg_b = p.Hkv * p.hgroups;
@@ -907,7 +907,33 @@ __global__ void __launch_bounds__(kMergeThreads, 2) decode_merge_kernel(const De
     r = hq % kDecHeadsPerSeg;
     return b * nseg_b + kvh * p.hgroups + hq / kDecHeadsPerSeg;
   };
-  for (long long base = 0; blockIdx.x + base * gridDim.x < rows; base += kMergeThreads) {
+  // Which rows were split, and over which CTAs, follows from the sequence
+  // lengths and the streaming kernel's plan alone (the same page prefix and
+  // equal shares of the unit line), so it is worked out before waiting for
+  // that kernel: the lengths are an input of the call, which the streaming
+  // kernel never writes, and were final before it started.
+  if (t < 32) {
+    const int per = (p.B + 31) / 32, b0 = t * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (b0 + i < p.B) local += dec_pages_of(p, b0 + i);
+    int incl = local;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (t >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int i = 0; i < per; ++i)
+      if (b0 + i < p.B) {
+        prefix[b0 + i] = run;
+        run += dec_pages_of(p, b0 + i);
+      }
+    if (t == 31) prefix[p.B] = incl;
+  }
+  __syncthreads();
+  const long long T = (long long)prefix[p.B] * nseg_b;   // the streaming kernel's unit line
+  const int C = (int)min((long long)p.parts, T);          // its CTAs with a non-empty share
+  auto build_list = [&](long long base) {
     if (t == 0) {
       nlist = 0;
       max_parts = 1;
@@ -915,17 +941,29 @@ __global__ void __launch_bounds__(kMergeThreads, 2) decode_merge_kernel(const De
     __syncthreads();
     const long long row = blockIdx.x + (base + t) * gridDim.x;
     if (row < rows) {
-      int r;
-      const int seg = seg_of((int)row, r);
-      // (a range outside this grid can only be left over from a call that
-      // stopped on a device error; it is skipped so no read leaves the slots)
-      const int2 info = p.ws_seg[seg];
-      if (info.x >= 0 && info.x <= info.y && info.y < p.parts) {
-        list[atomicAdd(&nlist, 1)] = (int)row;
-        atomicMax(&max_parts, info.y - info.x + 1);
+      const int b = (int)(row / p.Hq);
+      const int npg = prefix[b + 1] - prefix[b];
+      if (npg > 0) {   // (an empty sequence's rows were written by the streaming kernel)
+        int r;
+        const int seg_in_b = seg_of((int)row, r) - b * nseg_b;
+        const long long seg_u0 = (long long)prefix[b] * nseg_b + (long long)seg_in_b * npg;
+        const int first = dec_cta_of(seg_u0, T, C), last = dec_cta_of(seg_u0 + npg - 1, T, C);
+        if (first != last) {   // split: pieces in CTAs first..last
+          const int k = atomicAdd(&nlist, 1);
+          list[k] = (int)row;
+          range[k] = make_int2(first, last);
+          atomicMax(&max_parts, last - first + 1);
+        }
       }
     }
     __syncthreads();
+  };
+  build_list(0);
+  griddep_wait();   // the streaming kernel's partials
+  griddep_launch_dependents();
+
+  for (long long base = 0; blockIdx.x + base * gridDim.x < rows; base += kMergeThreads) {
+    if (base > 0) build_list(base);
     const int n = nlist;
     int gpr = 1;   // groups per row: a power of two with gpr * 4 >= parts
     while (gpr < kGroups && gpr * 4 < max_parts) gpr <<= 1;
@@ -939,7 +977,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2) decode_merge_kernel(const De
       if (k < n) {
         row_k = list[k];
         seg = seg_of(row_k, r);
-        const int2 info = p.ws_seg[seg];
+        const int2 info = range[k];
         // parts sub, sub + gpr, ... in batches of four whose loads are all
         // issued before any is used; every part holds at least one key, so
         // its LSE is finite (-inf marks a slot past the last part)
