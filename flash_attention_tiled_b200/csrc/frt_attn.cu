@@ -454,7 +454,10 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   const bool head_pairs = ((Hq / Hkv) % 2) == 0;
   const int blk_rows = head_pairs ? kPfBM : kPfRows;
   const int n_blocks = (Sq + blk_rows - 1) / blk_rows;
-  if (n_blocks > 65535) return FRT_ERR_UNSUPPORTED;
+  // work items: (sequence, query-head pair or head, query block)
+  const long long n_items = (long long)B * (head_pairs ? Hq / 2 : Hq) * n_blocks;
+  if (n_items > (1ll << 30)) return FRT_ERR_UNSUPPORTED;
+  if (n_items == 0) return FRT_OK;
   // Q, O (and contiguous K, V): 4D maps (d, token, head, batch) with the
   // tensors' own strides, one 128-row box per column half
   CUtensorMap tq, tk, tv, to;
@@ -499,6 +502,7 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.causal = causal;
   p.n_blocks = n_blocks;
   p.head_pairs = head_pairs ? 1 : 0;
+  p.n_items = (int)n_items;
   p.scale_log2 = scale * kLog2e;
   p.block_table = paged ? paged->block_table : nullptr;
   p.seq_lens = paged ? paged->seq_lens : nullptr;
@@ -506,7 +510,9 @@ frt_status launch_prefill(const void* q, const void* k, const void* v, void* o, 
   p.max_pages = paged ? paged->max_pages : 0;
   p.num_pages = paged ? paged->num_pages : 0;
   p.bad_row = paged ? paged->num_pages * Hkv * 16 : 0;
-  const dim3 grid((unsigned)(B * (head_pairs ? Hq / 2 : Hq)), (unsigned)n_blocks);
+  // persistent: one CTA per SM (the kernel holds a whole SM's shared memory),
+  // each walking its share of the items
+  const dim3 grid((unsigned)std::min<long long>(n_items, di->sm_count));
   auto* kernel = (paged == nullptr)
                      ? (D == 128 ? prefill_kernel<128, false> : prefill_kernel<64, false>)
                      : (D == 128 ? prefill_kernel<128, true> : prefill_kernel<64, true>);
