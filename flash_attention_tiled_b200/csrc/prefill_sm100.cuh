@@ -163,12 +163,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   using L = PrefillSmem<D>;
   constexpr int kHalves = L::kHalves;
   constexpr int kSlots = L::kSlots;
-  // Inputs may come from the kernel before this one in the stream: wait for
-  // it (a no-op unless launched as a programmatic dependent), then let the
-  // next kernel get scheduled as this grid's CTAs finish.
-  griddep_wait();
-  griddep_launch_dependents();
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -219,6 +213,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // The set-up above touches no global memory, so it may overlap the kernel
+  // before this one in the stream.  Inputs may come from that kernel: wait for
+  // it (a no-op unless launched as a programmatic dependent), then let the
+  // next kernel get scheduled as this grid's CTAs finish.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfRegsProducer));
@@ -382,21 +382,41 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return true;
       };
 
-      for (int r = 0; ok; ++r) {
-        const int w = prefill_item_index(r, cta, G);
-        if (w >= p.n_items) break;
-        const PrefillItem it = prefill_item<kPaged>(p, w);
-        if (it.n_kv == 0) continue;
+      // The items with a key tile, in this CTA's order, as their key-tile
+      // count (0: none left) and whether their last V tile has its tail
+      // zeroed.  The next one is decoded once the current one's first S pair
+      // is out, so the divisions stay off the issue path between two items.
+      int r_next = 0;
+      auto find_next = [&](int& n_kv_out, bool& tail_out) {
+        n_kv_out = 0;
+        tail_out = false;
+        for (;; ++r_next) {
+          const int w = prefill_item_index(r_next, cta, G);
+          if (w >= p.n_items) return;
+          const PrefillItem it = prefill_item<kPaged>(p, w);
+          if (it.n_kv > 0) {
+            n_kv_out = it.n_kv;
+            tail_out = it.v_tail_fill;
+            ++r_next;
+            return;
+          }
+        }
+      };
+      int n_kv, n_kv_next;
+      bool tail, tail_next;
+      find_next(n_kv, tail);
+      while (ok && n_kv > 0) {
         ok = mbar_wait(q_full, (uint32_t)(n_done & 1), &abort_flag);
-        if (ok) ok = issue_s(it.n_kv == 1);
-        for (int j = 0; j < it.n_kv && ok; ++j) {
-          if (j + 1 < it.n_kv) {
-            ok = issue_s(j + 2 == it.n_kv);
+        if (ok) ok = issue_s(n_kv == 1);
+        find_next(n_kv_next, tail_next);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          if (j + 1 < n_kv) {
+            ok = issue_s(j + 2 == n_kv);
             if (!ok) break;
           }
           // O_X += P_X(j).V_j as soon as P_X(j) is in shared memory
           ok = mbar_wait(&ring_full[slot], phase, &abort_flag);
-          if (ok && it.v_tail_fill && j == it.n_kv - 1) {
+          if (ok && tail && j == n_kv - 1) {
             ok = mbar_wait(v_tail, (uint32_t)(n_vt & 1), &abort_flag);
             ++n_vt;
           }
@@ -415,6 +435,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           next_slot();
         }
         ++n_done;
+        n_kv = n_kv_next;
+        tail = tail_next;
       }
       // every MMA of this thread must finish before tensor memory is freed
       tc_commit(mma_drain);
