@@ -590,14 +590,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++n_step;
       }
 
-      // ---- epilogue
-      if (ok && n_kv > 0)
-        ok = mbar_wait_warp(&pv_done[t], (uint32_t)((n_step - 1) & 1), &abort_flag);
+      // ---- epilogue (the item is decoded again while the last P.V runs)
       const PrefillItem it =
           prefill_item<kPaged>(p, prefill_item_index(opaque_int(r), cta, G));
       const int q0 = it.q_blk + t * it.dr;          // first query row of the tile
       const int hq = it.hq0 + t * it.dh;            // query head of the tile
       const int qi = q0 + r_row;                    // query index
+      if (ok && n_kv > 0)
+        ok = mbar_wait_warp(&pv_done[t], (uint32_t)((n_step - 1) & 1), &abort_flag);
       if (ok) {
         tc_fence_after();
         // a row that never saw a visible key (m_ref = -inf) gets o = 0 and
