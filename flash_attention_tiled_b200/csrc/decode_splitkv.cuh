@@ -553,20 +553,18 @@ decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // rows r8 (lo) and r8+8 (hi) of S^T as 16-bit pairs (heads 2qc,
             // 2qc+1): bf16, or f16 for the FP8 cache.  O is normalised by the
             // rounded weights that feed P.V; the LSE uses the exact ones
+            // (the rounded halves are added by the mixed-precision add)
             uint32_t lo, hi;
             if constexpr (kFp8) {
               lo = pack_f16x2(e[pg][0], e[pg][1]);
               hi = pack_f16x2(e[pg][2], e[pg][3]);
-              float a0, a1, b0, b1;
-              unpack_f16x2(lo, a0, a1);
-              unpack_f16x2(hi, b0, b1);
-              l_run[ht][0] += a0 + b0;
-              l_run[ht][1] += a1 + b1;
+              add_f16x2_to_f32(l_run[ht][0], l_run[ht][1], lo);
+              add_f16x2_to_f32(l_run[ht][0], l_run[ht][1], hi);
             } else {
               lo = pack_bf16x2(e[pg][0], e[pg][1]);
               hi = pack_bf16x2(e[pg][2], e[pg][3]);
-              l_run[ht][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
-              l_run[ht][1] += __uint_as_float(lo & 0xffff0000u) + __uint_as_float(hi & 0xffff0000u);
+              add_bf16x2_to_f32(l_run[ht][0], l_run[ht][1], lo);
+              add_bf16x2_to_f32(l_run[ht][0], l_run[ht][1], hi);
             }
             le_run[ht][0] += e[pg][0] + e[pg][2];
             le_run[ht][1] += e[pg][1] + e[pg][3];

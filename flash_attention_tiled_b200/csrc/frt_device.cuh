@@ -132,6 +132,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// lo += the low bf16 half of w, hi += its high half, each converted to fp32
+// inside the add (the mixed-precision add of sm_100: no separate unpack).
+__device__ __forceinline__ void add_bf16x2_to_f32(float& lo, float& hi, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+      : "+f"(lo), "+f"(hi)
+      : "r"(w));
+}
+
+// The same for an f16 pair.
+__device__ __forceinline__ void add_f16x2_to_f32(float& lo, float& hi, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %0;\n\tadd.rn.f32.f16 %1, h, %1;\n\t}"
+      : "+f"(lo), "+f"(hi)
+      : "r"(w));
+}
+
 // 16-byte store to shared memory at a 32-bit shared-window address.
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {

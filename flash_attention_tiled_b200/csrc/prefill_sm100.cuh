@@ -556,7 +556,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         {
           const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
           const uint64_t ref2 = f2_pack(neg_ref, neg_ref);
-          uint64_t es0 = 0, es1 = 0, rs0 = 0, rs1 = 0;   // packed partial sums (0.0f pairs)
+          uint64_t es0 = 0, es1 = 0;   // exact partial sums, packed (0.0f pairs)
+          float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;   // rounded partial sums
 #pragma unroll
           for (int c8 = 0; c8 < kPfBN; c8 += 8) {
             uint32_t wv[4];
@@ -568,19 +569,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               e0 = fast_exp2(x0);
               e1 = fast_exp2(x1);
               wv[q] = pack_bf16x2(e0, e1);
-              const uint64_t wr = f2_pack(__uint_as_float(wv[q] << 16),
-                                          __uint_as_float(wv[q] & 0xffff0000u));
-              if (q & 1) { es1 = f2_add(es1, f2_pack(e0, e1)); rs1 = f2_add(rs1, wr); }
-              else       { es0 = f2_add(es0, f2_pack(e0, e1)); rs0 = f2_add(rs0, wr); }
+              // the rounded weights are added straight from their bf16 halves
+              if (q & 1) {
+                es1 = f2_add(es1, f2_pack(e0, e1));
+                add_bf16x2_to_f32(rs2, rs3, wv[q]);
+              } else {
+                es0 = f2_add(es0, f2_pack(e0, e1));
+                add_bf16x2_to_f32(rs0, rs1, wv[q]);
+              }
             }
             const int chunk = c8 >> 3, h = chunk >> 3, ch = chunk & 7;
             st_shared_v4(row_addr + h * L::kHalfBytes + ((ch ^ sw) << 4), wv[0], wv[1], wv[2],
                          wv[3]);
           }
-          float a2, b2, c2, d2;
-          f2_unpack(f2_add(rs0, rs1), a2, b2);
+          float c2, d2;
           f2_unpack(f2_add(es0, es1), c2, d2);
-          l_sum += a2 + b2;
+          l_sum += (rs0 + rs1) + (rs2 + rs3);
           l_exact += c2 + d2;
         }
         tc_wait_st();   // O rescale stores, if any, before PV_t(j) may run
