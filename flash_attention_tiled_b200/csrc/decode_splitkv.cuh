@@ -50,21 +50,26 @@ namespace frt {
 constexpr int kDecPage = 16;          // tokens per page (one MMA K-step)
 // Consumer warps per CTA (a power of two) and the pages each takes per
 // stage.  With one 8-head tile the consumers, not HBM, set the pace with two
-// warps, so there are four: two pages each for the FP8 cache (a stage of 8
-// FP8 pages is 32 KB), one each for bf16 (4 pages, 32 KB).  Otherwise two
-// warps of two pages.
+// warps, so there are four of one page each (a stage of 4 pages: 32 KB for
+// bf16, 16 KB for FP8).  Otherwise two warps of two pages.
+// CTAs per SM and ring size: the FP8 cache with one head tile is
+// consumer-latency-bound, so its SMs take three CTAs of a 48 KB ring (the
+// kernel fits in 122 registers) instead of two of 96 KB; measured on B200:
+// 256k decode 52.5 -> 51.4 us, the paged B4 one unchanged.
 template <bool kFp8, int kHT>
 struct DecodeCfg {
   static constexpr int kWarps = (kHT == 1) ? 4 : 2;
-  static constexpr int kPagesPerWarp = (kHT == 1 && !kFp8) ? 1 : 2;
+  static constexpr int kPagesPerWarp = (kHT == 1) ? 1 : 2;
   static constexpr int kStagePages = kWarps * kPagesPerWarp;
   static constexpr int kThreads = 32 * (kWarps + 1);
+  static constexpr int kCtasPerSm = (kFp8 && kHT == 1) ? 3 : 2;
+  static constexpr int kRingBytes = (kFp8 && kHT == 1 ? 48 : 96) * 1024;
 };
-// Up to two CTAs share an SM: two independent TMA rings per SM keep more
-// page copies in flight than one ring twice as deep.  The default grid aims
-// at about 18 MiB of page copies in flight over the whole GPU (192 CTAs of
-// a 96 KB ring); measured on B200, fewer starve HBM of requests and more
-// (two rings on every SM, 28 MiB) read measurably slower.
+// bf16 cache: up to two CTAs share an SM: two independent TMA rings per SM
+// keep more page copies in flight than one ring twice as deep.  The default
+// grid aims at about 18 MiB of page copies in flight over the whole GPU (192
+// CTAs of a 96 KB ring); measured on B200, fewer starve HBM of requests and
+// more (two rings on every SM, 28 MiB) read measurably slower.
 constexpr int kDecCtasPerSm = 2;
 constexpr long long kDecInFlightBytes = 18ll << 20;
 constexpr int kDecHeadsPerSeg = 16;   // MMA M dimension
@@ -108,7 +113,7 @@ struct DecodeSmem {
   static constexpr int kBoxBytes = kDecPage * 128;                    // 16 rows x 128 bytes
   static constexpr int kPageBytes = kDecPage * D * (kFp8 ? 1 : 2);   // K or V of one page
   static constexpr int kStageBytes = Cfg::kStagePages * 2 * kPageBytes; // K+V of a stage
-  static constexpr int kStages = (96 * 1024) / kStageBytes;           // 96 KB ring
+  static constexpr int kStages = Cfg::kRingBytes / kStageBytes;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // cross-warp combine: one warp's register state in fragment order
   // (D/16 m-tiles x kHT head tiles x 4 accumulators, then m, l, l_exact for
@@ -128,7 +133,7 @@ struct DecodeSmem {
   static_assert(kBarOff % 8 == 0, "mbarriers need 8-byte alignment");
   // per SM: 228 KB, of which each CTA also reserves 1 KB (static shared
   // variables live in the slack below)
-  static_assert(kDecCtasPerSm * (kBytes + 1024 + 64) <= 228 * 1024, "shared memory budget");
+  static_assert(Cfg::kCtasPerSm * (kBytes + 1024 + 64) <= 228 * 1024, "shared memory budget");
 };
 
 // Pages of sequence b (seq_len clamped to [0, max_pages * 16]).
@@ -178,7 +183,7 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int 
 // kCluster: cluster mode (see the top of this file): contiguous bf16 cache,
 // launched with a cluster of C CTAs per segment; nothing goes to a workspace.
 template <int D, int kHT, bool kFp8, bool kCluster = false>
-__global__ void __launch_bounds__(DecodeCfg<kFp8, kHT>::kThreads, kDecCtasPerSm)
+__global__ void __launch_bounds__(DecodeCfg<kFp8, kHT>::kThreads, DecodeCfg<kFp8, kHT>::kCtasPerSm)
 decode_splitkv_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   static_assert(!(kCluster && kFp8), "cluster mode reads a bf16 cache");

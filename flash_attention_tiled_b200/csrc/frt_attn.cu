@@ -258,12 +258,12 @@ frt_status launch_decode(const void* q, const void* k_base, const void* v_base,
     // bf16 cache: enough partitions for kDecInFlightBytes of page copies in
     // flight (192 on a 148-SM B200; measured faster than one or two per SM).
     // FP8 cache: its consumer warps, not HBM, set the pace, so every SM gets
-    // two partitions (measured on B200: 11 % faster than the bf16 plan).
+    // as many partitions as it holds CTAs (three with one head tile, else two).
+    const long long per_sm = !fp8 ? kDecCtasPerSm
+                             : (g <= 8 ? DecodeCfg<true, 1>::kCtasPerSm : DecodeCfg<true, 2>::kCtasPerSm);
     const long long ring = (D == 128) ? DecodeSmem<128>::kRingBytes : DecodeSmem<64>::kRingBytes;
-    const long long want = fp8 ? (long long)kDecCtasPerSm * di->sm_count
-                               : (kDecInFlightBytes + ring - 1) / ring;
-    parts = (int)std::min<long long>(std::max<long long>(want, di->sm_count),
-                                     (long long)kDecCtasPerSm * di->sm_count);
+    const long long want = fp8 ? per_sm * di->sm_count : (kDecInFlightBytes + ring - 1) / ring;
+    parts = (int)std::min<long long>(std::max<long long>(want, di->sm_count), per_sm * di->sm_count);
   }
   const DecodeWorkspace wl = decode_ws_layout(parts, segments, D);
   if (query) {

@@ -285,8 +285,9 @@ FRT_API frt_status frt_attn_fwd_strided(const void* q, const void* k, const void
  * of KV head h stands for code * k_scale[h] (keys) or code * v_scale[h]
  * (values); every other argument means what it means for
  * frt_attn_decode_paged, and the workspace size query is the same, except
- * that num_splits = 0 means two partitions per SM (296 on a 148-SM B200):
- * with one byte per element the kernel's arithmetic, not HBM, sets its pace.
+ * that num_splits = 0 means three partitions per SM when a KV head serves
+ * at most 8 query heads (444 on a 148-SM B200), else two: with one byte per
+ * element the kernel's arithmetic, not HBM, sets its pace.
  *   k_scale, v_scale  [Hkv] fp32 on the device, finite, 4-byte aligned
  *   D                 128 only (FRT_ERR_UNSUPPORTED otherwise)
  * The kernel converts codes to f16 (exact), multiplies q.k in f16 with fp32
