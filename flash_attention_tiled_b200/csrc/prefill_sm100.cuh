@@ -10,18 +10,19 @@
 // optimisation".  Key tiles that the causal mask hides completely are never
 // loaded or multiplied.
 //
-// One CTA owns two 128-row query tiles A and B that share every K/V tile.
+// A work item is two 128-row query tiles A and B that share every K/V tile.
 // When a KV head serves an even number of query heads (GQA with g even, MQA)
 // the tiles are the same 128 rows of two query heads of one KV head, so each
 // K/V tile staged in shared memory serves two heads of its group (the MQA/GQA
 // head sharing of the "FlashRT-HF-kernels" page); otherwise (g odd, e.g. MHA)
-// they are rows 0-127 and 128-255 of a 256-row block of one head.  Tensor memory holds
-// S_A, S_B (128 fp32 columns each) and O_A, O_B (D columns each).  P_X is
-// written as bf16 into its own shared-memory tile (the A operand of
-// O_X += P_X.V), so S_X is free as soon as the softmax has read it: S_X(j+1)
-// is computed while the softmax of tile j is still busy.
+// they are rows 0-127 and 128-255 of a 256-row block of one head.  The kernel
+// is persistent: one CTA per SM walks its items (see prefill_kernel).
+// Tensor memory holds S_A, S_B (128 fp32 columns each) and O_A, O_B (D
+// columns each).  P_X is written as bf16 into its own shared-memory tile (the
+// A operand of O_X += P_X.V), so S_X is free as soon as the softmax has read
+// it: S_X(j+1) is computed while the softmax of tile j is still busy.
 // Roles (12 warps):
-//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles into a
+//   warp 0      TMA producer: per item Q_A and Q_B, then K and V tiles into a
 //               ring of shared-memory slots (128-byte swizzled), in the
 //               order the MMA warp uses them (K0, K1, V0, K2, V1, ...).
 //   warp 1      allocates tensor memory and issues every MMA from one
@@ -31,7 +32,7 @@
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query row
 //               per thread (= one TMEM lane); exp2 domain (scale*log2(e)
 //               folded in); then the epilogue (O / l -> bf16 -> shared memory
-//               -> TMA store, and the LSE).
+//               (P's slot) -> TMA store, and the LSE).
 // The producer/MMA warpgroup gives registers to the two softmax warpgroups
 // (setmaxnreg): 128 x 88 + 256 x 208 = 384 x 168 registers, the launch's pool.
 // Rescaling is lazy: the exponent reference only moves when the row max grows
