@@ -22,7 +22,8 @@
 // launched as a programmatic dependent, so it is resident and waiting when
 // the streaming kernel ends.  No CTA ever waits for another.
 //
-// Inside a CTA (two per SM): warp 0 streams pages into a ring of
+// Inside a CTA (two per SM; three for the FP8 cache with one head tile):
+// warp 0 streams pages into a ring of
 // shared-memory stages with TMA (one 128-byte swizzled box per page and
 // matrix, one mbarrier per stage), looking pages up in the block table;
 // warps 1..W (DecodeCfg) each take one or two pages of every stage and compute
